@@ -1,0 +1,235 @@
+/*
+ * svdq.h -- C ABI of the B200 (sm_100a) SVDQuant W4A4 + low-rank linear layer.
+ *
+ * The layer (SVDQuant: Absorbing Outliers by Low-Rank Components for 4-Bit
+ * Diffusion Models; paperlayer.ai summary of arXiv 2411.05007v4, §4.2 and §4.3):
+ *
+ *   Y = Q4(X diag(lam)^-1) Q4(R)^T * alpha_w  +  (X diag(lam)^-1 L1) L2  +  b
+ *
+ * X is M x K (tokens x in-features), W is N x K (out x in, the PyTorch
+ * Linear.weight layout), b is N.  A 16-bit rank-r branch L1 (K x r), L2 (r x N)
+ * from the SVD of the smoothed weight W_hat = W diag(lam) takes the outliers,
+ * and the residual R = W_hat - (L1 L2)^T is quantized to NVFP4: E2M1 codes
+ * with one E4M3 scale per 16 consecutive elements along K (App. D).  The
+ * runtime is two kernels (§4.3, Fig. 6): the activation kernel quantizes X and
+ * computes the down-projection from the same read of X; the GEMM kernel folds
+ * the up-projection into its 4-bit accumulator.
+ *
+ * Conventions for every call:
+ *  - Element types: bf16 values are passed as their uint16 bit patterns;
+ *    fp32 as float.  All matrices are row-major with the last index
+ *    contiguous.
+ *  - "host" pointers are ordinary CPU memory (pinned memory makes the copies
+ *    of svdq_forward_host asynchronous); "device" pointers are global memory of
+ *    the current CUDA device and must be 16-byte aligned.
+ *  - Ownership: the caller owns every buffer it passes and keeps device
+ *    buffers alive until the work queued on the stream has finished.  The
+ *    library owns the svdq_weights handle and the device memory inside it;
+ *    svdq_weights_destroy frees both.
+ *  - Streams: `stream` is a cudaStream_t passed as void* (NULL = the legacy
+ *    default stream).  Runtime calls only enqueue work; they do not
+ *    synchronize.  Weight preparation and LoRA attachment synchronize.
+ *  - Errors: every call validates its arguments on the host before touching
+ *    the GPU and returns a status; svdq_last_error() gives a message for the
+ *    last failure on the calling thread.  Device-side failures (a wait that ran
+ *    past its time limit) are recorded in a device error word that
+ *    svdq_check_device_errors() reads.
+ *  - Shape limits: K % 64 == 0; N % 16 == 0; 1 <= M; rank + LoRA ranks <= 128.
+ *    The device must be sm_100 (B200).
+ */
+#ifndef SVDQ_H_
+#define SVDQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct svdq_weights svdq_weights; /* opaque, library-owned */
+
+typedef enum {
+  SVDQ_OK = 0,
+  SVDQ_ERR_INVALID_ARG = 1,        /* a null pointer, bad shape or misaligned pointer */
+  SVDQ_ERR_UNSUPPORTED_DEVICE = 2, /* the current device is not sm_100 */
+  SVDQ_ERR_CUDA = 3,               /* a CUDA runtime/driver call failed */
+  SVDQ_ERR_OOM = 4,                /* device or host allocation failed */
+  SVDQ_ERR_TIMEOUT = 5,            /* a kernel wait passed its time limit */
+  SVDQ_ERR_DEVICE_CHECK = 6        /* a kernel's own bounds/launch check failed */
+} svdq_status;
+
+/* Options of the offline weight transform. */
+typedef struct {
+  float alpha;        /* smoothing migration strength (App. D); default 0.5 */
+  int rank;           /* low-rank branch rank r (§4.2: 16 or 32); default 32 */
+  int power_iters;    /* subspace iterations of the randomized SVD; default 4 */
+  int oversample;     /* extra columns of the random subspace; default 16 */
+  uint64_t seed;      /* seed of the random starting subspace; default 0 */
+  int keep_residual;  /* nonzero: keep a host copy of R/alpha_w for export */
+} svdq_prepare_opts;
+
+/* Fills *opts with the defaults above. */
+void svdq_prepare_opts_default(svdq_prepare_opts* opts);
+
+/*
+ * Offline weight transform (§4.2 and App. D): smoothing factors
+ * lam_j = act_absmax_j^alpha / max_n |W_nj|^(1-alpha) (lam_j = 1 when either
+ * maximum is 0), W_hat = W diag(1/fp32(1/lam)), a top-r SVD of W_hat by
+ * randomized subspace iteration on the host, 16-bit factors
+ * L1' = bf16(diag(inv_lam) L1) and L2 = bf16(V_r^T), the residual
+ * R = W_hat - (diag(1/inv_lam) L1' L2)^T, the power-of-two factor
+ * alpha_w = 2^ceil(log2(max|R| / 2688)), and the NVFP4 codes of R/alpha_w
+ * (computed on the device).
+ *   W_bf16      host, N x K bf16 (out x in)
+ *   act_absmax  host, K floats: per-input-channel max |x| over calibration data
+ *   bias_bf16   host, N bf16, or NULL for no bias
+ *   opts        NULL for the defaults
+ *   out         receives the new handle (NULL on failure)
+ * Synchronizes `stream`.
+ */
+svdq_status svdq_prepare_weights(const uint16_t* W_bf16, const float* act_absmax,
+                                 const uint16_t* bias_bf16, int N, int K,
+                                 const svdq_prepare_opts* opts, void* stream,
+                                 svdq_weights** out);
+
+/*
+ * Builds a handle from a given split (the second half of
+ * svdq_prepare_weights): alpha_w is chosen from R as above and R/alpha_w is
+ * quantized on the device.  This lets a caller supply factors computed
+ * elsewhere (for instance an exact SVD).
+ *   inv_lam   host, K floats (the runtime activation multipliers 1/lam)
+ *   L1p_bf16  host, K x rank bf16 (L1' = diag(inv_lam) L1), or NULL if rank == 0
+ *   L2_bf16   host, rank x N bf16, or NULL if rank == 0
+ *   R         host, N x K floats: the residual (not yet divided by alpha_w)
+ *   bias      host, N floats, or NULL
+ * Synchronizes `stream`.
+ */
+svdq_status svdq_weights_from_factors(int N, int K, int rank, const float* inv_lam,
+                                      const uint16_t* L1p_bf16, const uint16_t* L2_bf16,
+                                      const float* R, const float* bias, void* stream,
+                                      svdq_weights** out);
+
+/*
+ * LoRA without re-quantization (§2; §5.2 and Fig. 9: the low-rank branch
+ * absorbs the LoRA by growing its rank).  Appends A as new columns of L1'
+ * (A acts on the unsmoothed X, so it is not scaled by inv_lam) and
+ * bf16(scale * B) as new rows of L2.  The 4-bit codes, scales and alpha_w are
+ * not touched.
+ *   A_bf16  host, K x r_l bf16 (LoRA down)
+ *   B_bf16  host, r_l x N bf16 (LoRA up)
+ * Synchronizes `stream`.
+ */
+svdq_status svdq_attach_lora(svdq_weights* w, const uint16_t* A_bf16, const uint16_t* B_bf16,
+                             int r_l, float scale, void* stream);
+
+/*
+ * Kernel 1, activation side (§4.3: the down-projection is fused into the
+ * quantization kernel so X is read once).  For each row m and group of 16
+ * along K: x_hat = fp32(x * inv_lam_j); amax = max|x_hat|;
+ * s = E4M3_rne_satfinite(fp32(amax/6)); codes = E2M1_rne_satfinite(
+ * fp32(x_hat * fp32(1/s))) (all +0 when s decodes to 0; a code that rounds to
+ * magnitude 0 is stored as +0).  In the same pass T = X L1' (fp32 on the
+ * tensor cores) is written as an unevaluated bf16 pair T = T_hi + T_lo.
+ *   X_bf16  device, M x K bf16
+ *   xq      device, M x K/2 bytes: two codes per byte, element 2i in the low nibble
+ *   xsf     device, svdq_act_sf_bytes(M, K) bytes: E4M3 scales in the Blackwell
+ *           block-scale layout (128-row x 4-column atoms of 512 bytes, K-atoms
+ *           fastest; inside an atom row m, column j is byte
+ *           (m%32)*16 + (m/32)*4 + j; padded rows get scale 0)
+ *   T       device, svdq_lowrank_bytes(w, M) bytes: M rows of 2*r_pad bf16 where,
+ *           for each 16-wide chunk c of the rank, columns [32c, 32c+16) hold T_hi
+ *           and [32c+16, 32c+32) hold T_lo.  May be NULL when the rank is 0.
+ */
+svdq_status svdq_quantize_act_lowrank_down(const svdq_weights* w, const void* X_bf16, int M,
+                                           void* xq, void* xsf, void* T, void* stream);
+
+/*
+ * Kernel 2, the 4-bit GEMM with the up-projection folded in (§4.3):
+ * Y = bf16_rne(alpha_w * (sum_k deq(xq) deq(wq) + (T_hi + T_lo) (L2 / alpha_w)) + b),
+ * accumulated in fp32 in tensor memory.
+ *   xq, xsf, T  as written by svdq_quantize_act_lowrank_down for the same M
+ *   Y_bf16      device, M x N bf16
+ */
+svdq_status svdq_linear_w4a4(const svdq_weights* w, const void* xq, const void* xsf,
+                             const void* T, int M, void* Y_bf16, void* stream);
+
+/*
+ * Both kernels back to back.  `workspace` is device memory of at least
+ * svdq_forward_workspace_bytes(w, M) bytes holding xq, xsf and T.
+ */
+svdq_status svdq_forward(const svdq_weights* w, const void* X_bf16, int M, void* Y_bf16,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * svdq_forward with host input and output: copies X (host, M x K bf16) into
+ * the workspace, runs both kernels and copies Y (M x N bf16) back into Y_host,
+ * all enqueued on `stream` (no synchronization).  `workspace` is device memory
+ * of at least svdq_forward_host_workspace_bytes(w, M) bytes.
+ */
+svdq_status svdq_forward_host(const svdq_weights* w, const void* X_host, int M, void* Y_host,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/* Sizes in bytes. */
+size_t svdq_act_codes_bytes(int M, int K);                 /* M * K / 2 */
+size_t svdq_act_sf_bytes(int M, int K);                    /* ceil(M/128)*128 * K/16 */
+size_t svdq_lowrank_bytes(const svdq_weights* w, int M);   /* M * 2 * r_pad * 2 */
+size_t svdq_forward_workspace_bytes(const svdq_weights* w, int M);
+size_t svdq_forward_host_workspace_bytes(const svdq_weights* w, int M);
+
+/* Shape of a handle: rank counts the SVD rank plus attached LoRA ranks, r_pad
+ * is that rounded up to a multiple of 16 (the width of T's hi and lo parts). */
+svdq_status svdq_weights_info(const svdq_weights* w, int* N, int* K, int* rank, int* r_pad,
+                              float* alpha_w);
+
+/*
+ * Copies the handle's contents to host memory (tests and inspection).  Any
+ * output may be NULL to skip it.
+ *   codes     N x K/2 bytes        sf      svdq_act_sf_bytes(N, K) bytes (atom layout)
+ *   L1p_bf16  K x rank bf16        L2_bf16 rank x N bf16 (not divided by alpha_w)
+ *   inv_lam   K floats             bias    N floats
+ *   residual  N x K floats R/alpha_w; only if the handle kept it, else
+ *             SVDQ_ERR_INVALID_ARG
+ * Synchronizes the device.
+ */
+svdq_status svdq_weights_export(const svdq_weights* w, uint8_t* codes, uint8_t* sf,
+                                uint16_t* L1p_bf16, uint16_t* L2_bf16, float* inv_lam,
+                                float* bias, float* residual);
+
+/* Frees the handle and its device memory (NULL is allowed). */
+svdq_status svdq_weights_destroy(svdq_weights* w);
+
+/*
+ * Time limit, in nanoseconds, of every wait inside the kernels (default
+ * 2e9).  When a wait passes it the kernel records SVDQ_ERR_TIMEOUT in the
+ * device error word, skips its remaining work and exits cleanly.
+ */
+void svdq_set_wait_limit_ns(uint64_t ns);
+
+/*
+ * Synchronizes `stream`, then reads and clears the current device's error
+ * word: SVDQ_OK, SVDQ_ERR_TIMEOUT or SVDQ_ERR_DEVICE_CHECK.
+ */
+svdq_status svdq_check_device_errors(void* stream);
+
+/*
+ * Test hook for the bounded waits: launches the activation kernel with a
+ * wait that nothing completes (its pipeline barrier expects one more arrival
+ * than it gets), so that the wait runs out after svdq_set_wait_limit_ns and
+ * the kernel exits with SVDQ_ERR_TIMEOUT in the device error word.  Buffers
+ * as for svdq_quantize_act_lowrank_down.
+ */
+svdq_status svdq_debug_launch_stalled_act(const svdq_weights* w, const void* X_bf16, int M,
+                                          void* xq, void* xsf, void* T, void* stream);
+
+/* Message for the last failed call on this thread ("" if none). */
+const char* svdq_last_error(void);
+
+/* Library version string. */
+const char* svdq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SVDQ_H_ */

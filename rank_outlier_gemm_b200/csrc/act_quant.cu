@@ -1,0 +1,320 @@
+// Kernel 1: activation quantization with the low-rank down-projection fused in.
+//
+// SVDQuant §4.3 (Nunchaku, Fig. 6): the down-projection shares the activation
+// read with the quantization kernel.  One CTA owns 128 rows of X and a slice of
+// K; S CTAs of a thread-block cluster split K and reduce their partial
+// T = X L1' through distributed shared memory.
+//
+// Per 64-column K tile (one TMA box, 128-byte swizzled rows):
+//   warp 0     TMA producer: X tile [128 x 64] bf16 and L1'^T tile [r_pad x 64]
+//   warp 1     tcgen05.mma kind::f16 (M=128, N=r_pad, K=16 x 4) into TMEM, same
+//              shared-memory X tile as the quantizers read
+//   warps 2-5  thread = row: smoothing multiply, per-16 amax, E4M3 scale,
+//              E2M1 codes; 32 code bytes and one 4-byte scale word per row
+// After the K loop the quantizer warps move T from TMEM to shared memory, the
+// cluster syncs, each CTA sums its share of rows over all S partials and writes
+// T as a bf16 hi/lo pair.
+#include <algorithm>
+
+#include "nvfp4.cuh"
+#include "svdq_internal.h"
+
+namespace svdq {
+namespace {
+
+using namespace dev;
+
+constexpr int kStages = 4;
+constexpr int kThreads = 192;
+constexpr int kXTile = 128 * 128;  // 128 rows x 64 bf16
+
+struct K1Params {
+  int M, K, r_pad, kt_total, splits;
+  const float* inv_lam;
+  uint8_t* xq;
+  uint8_t* xsf;
+  uint16_t* T;
+  int* err;
+  uint64_t wait_ns;
+  int stall;
+  uint32_t l1_tile;    // r_pad * 128 bytes
+  uint32_t tmem_cols;
+};
+
+struct K1Shared {
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t tfull;
+  uint64_t never;
+  uint32_t tmem_base;
+  int abort;
+};
+
+// Waits for a phase with a time limit only (used when draining after an abort).
+__device__ __noinline__ bool wait_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer() - t0 > limit_ns) return false;
+  }
+  return true;
+}
+
+__device__ __forceinline__ void bar_sync_quant() {
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(kThreads) act_quant_lowrank_kernel(
+    const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_l1,
+    const K1Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* xs = smem;
+  uint8_t* l1s = smem + kStages * kXTile;
+  K1Shared* sh = reinterpret_cast<K1Shared*>(l1s + kStages * p.l1_tile);
+  float* red = reinterpret_cast<float*>(smem);  // reuses the stage buffers after the K loop
+  const int red_stride = p.r_pad + 4;
+
+  const uint32_t warp = warp_id(), lane = lane_id();
+  const int mb = blockIdx.x;
+  const int m0 = mb * 128;
+  const int split = static_cast<int>(blockIdx.y);
+  const int base = p.kt_total / p.splits, rem = p.kt_total % p.splits;
+  const int nt = base + (split < rem ? 1 : 0);
+  const int t0 = split * base + min(split, rem);
+  const bool lowrank = p.r_pad > 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sh->full[s], 1);
+      mbar_init(&sh->empty[s], 4 + (lowrank ? 1 : 0));
+    }
+    mbar_init(&sh->tfull, 1);
+    mbar_init(&sh->never, 1);
+    sh->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1 && lowrank) {
+    tmem_alloc(&sh->tmem_base, p.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const WaitCtl wc{p.err, p.wait_ns, &sh->abort};
+  const uint32_t tmem = lowrank ? sh->tmem_base : 0u;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&map_x);
+      if (lowrank) tma_prefetch_desc(&map_l1);
+      const uint32_t bytes = kXTile + (lowrank ? p.l1_tile : 0u);
+      int issued = 0;
+      for (int i = 0; i < nt; ++i) {
+        const int s = i % kStages;
+        const uint32_t ph = (i / kStages) & 1;
+        if (!wait_bounded(&sh->empty[s], ph ^ 1, wc)) break;
+        mbar_arrive_expect_tx(&sh->full[s], bytes);
+        const int k0 = (t0 + i) * 64;
+        tma_load_2d(xs + s * kXTile, &map_x, &sh->full[s], k0, m0);
+        if (lowrank) tma_load_2d(l1s + s * p.l1_tile, &map_l1, &sh->full[s], k0, 0);
+        issued = i + 1;
+      }
+      if (sh->abort) {  // let copies in flight land before the buffers are reused
+        for (int i = max(0, issued - kStages); i < issued; ++i)
+          wait_drain(&sh->full[i % kStages], (i / kStages) & 1, p.wait_ns);
+      }
+    }
+  } else if (warp == 1) {
+    if (lowrank && lane == 0) {
+      const uint32_t idesc = idesc_bf16(128, p.r_pad);
+      for (int i = 0; i < nt; ++i) {
+        const int s = i % kStages;
+        const uint32_t ph = (i / kStages) & 1;
+        if (!wait_bounded(&sh->full[s], ph, wc)) break;
+        tc_fence_after();
+        const uint32_t xa = smem_u32(xs + s * kXTile);
+        const uint32_t la = smem_u32(l1s + s * p.l1_tile);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          mma_bf16(tmem, desc_kmajor_sw128(xa + 32 * k), desc_kmajor_sw128(la + 32 * k), idesc,
+                   (i | k) != 0);
+        mma_commit(&sh->empty[s]);
+      }
+      mma_commit(&sh->tfull);
+    }
+  } else {
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int row = q * 32 + lane;
+    const int m = m0 + row;
+    if (p.stall) wait_bounded(&sh->never, 0, wc);
+    for (int i = 0; i < nt; ++i) {
+      const int s = i % kStages;
+      const uint32_t ph = (i / kStages) & 1;
+      if (!wait_bounded(&sh->full[s], ph, wc)) break;
+      const uint8_t* xrow = xs + s * kXTile + row * 128;
+      const int kt = t0 + i;
+      const int k0 = kt * 64;
+      uint32_t codes[8];
+      uint32_t sc = 0;
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        // 128-byte swizzle: 16-byte chunk c of row r sits at chunk c ^ (r % 8).
+        const uint4 c0 = *reinterpret_cast<const uint4*>(xrow + (((2 * g) ^ (row & 7)) << 4));
+        const uint4 c1 = *reinterpret_cast<const uint4*>(xrow + (((2 * g + 1) ^ (row & 7)) << 4));
+        const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        const float4* il = reinterpret_cast<const float4*>(p.inv_lam + k0 + 16 * g);
+        const float4 i0 = __ldg(il), i1 = __ldg(il + 1), i2 = __ldg(il + 2), i3 = __ldg(il + 3);
+        const float inv[16] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w,
+                               i2.x, i2.y, i2.z, i2.w, i3.x, i3.y, i3.z, i3.w};
+        float v[16];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          v[2 * j] = __fmul_rn(__uint_as_float(w[j] << 16), inv[2 * j]);
+          v[2 * j + 1] = __fmul_rn(__uint_as_float(w[j] & 0xFFFF0000u), inv[2 * j + 1]);
+        }
+        const Fp4Group gq = nvfp4_encode16(v);
+        codes[2 * g] = gq.lo;
+        codes[2 * g + 1] = gq.hi;
+        sc |= gq.scale << (8 * g);
+      }
+      if (m < p.M) {
+        uint4* dst = reinterpret_cast<uint4*>(p.xq + static_cast<size_t>(m) * (p.K / 2) + k0 / 2);
+        dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+        dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+      }
+      const size_t atom = static_cast<size_t>(mb) * p.kt_total + kt;
+      *reinterpret_cast<uint32_t*>(p.xsf + atom * 512 + (row & 31) * 16 + (row >> 5) * 4) = sc;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->empty[s]);
+    }
+    if (lowrank) {
+      bar_sync_quant();  // every quantizer is done with the stage buffers
+      if (!sh->abort && wait_bounded(&sh->tfull, 0, wc)) {
+        tc_fence_after();
+        float* dst = red + row * red_stride;
+        for (int c = 0; c < p.r_pad; c += 16) {
+          uint32_t r[16];
+          tmem_ld_x16(tmem + (static_cast<uint32_t>(q * 32) << 16) + c, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; j += 4)
+            *reinterpret_cast<float4*>(dst + c + j) =
+                make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]),
+                            __uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
+        }
+      }
+    }
+  }
+
+  // ---- cluster-wide reduction of the partial T over the K splits
+  tc_fence_before();
+  cluster_sync_all();
+  if (lowrank && !sh->abort) {
+    const int rows_per = (128 + p.splits - 1) / p.splits;
+    const int r_lo = split * rows_per;
+    const int r_hi = min(128, r_lo + rows_per);
+    const int c4n = p.r_pad / 4;
+    const uint32_t red_addr = smem_u32(red);
+    for (int it = threadIdx.x; it < (r_hi - r_lo) * c4n; it += kThreads) {
+      const int rr = r_lo + it / c4n;
+      const int c = (it % c4n) * 4;
+      const int m = m0 + rr;
+      if (m >= p.M) continue;
+      const uint32_t off = static_cast<uint32_t>((rr * red_stride + c) * 4);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int qr = 0; qr < p.splits; ++qr) {
+        const float4 v = ld_dsmem_f4(mapa_shared(red_addr + off, qr));
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+      }
+      const float a[4] = {acc.x, acc.y, acc.z, acc.w};
+      uint16_t hi[4], lo[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const __nv_bfloat16 h = __float2bfloat16_rn(a[j]);
+        hi[j] = __bfloat16_as_ushort(h);
+        lo[j] = __bfloat16_as_ushort(__float2bfloat16_rn(a[j] - __bfloat162float(h)));
+      }
+      uint16_t* trow = p.T + static_cast<size_t>(m) * (2 * p.r_pad) + 32 * (c / 16) + (c % 16);
+      *reinterpret_cast<uint2*>(trow) =
+          make_uint2(hi[0] | (uint32_t(hi[1]) << 16), hi[2] | (uint32_t(hi[3]) << 16));
+      *reinterpret_cast<uint2*>(trow + 16) =
+          make_uint2(lo[0] | (uint32_t(lo[1]) << 16), lo[2] | (uint32_t(lo[3]) << 16));
+    }
+  }
+  cluster_sync_all();  // peers are done reading this CTA's partial
+
+  if (warp == 1 && lowrank) {
+    if (lane == 0) wait_drain(&sh->tfull, 0, p.wait_ns);  // every MMA has retired
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, p.tmem_cols);
+  }
+}
+
+int auto_splits(int mblocks, int kt_total) {
+  // Aim for about two CTAs per SM (148 SMs) while keeping >= 4 K tiles per CTA.
+  int s = (2 * 148 + mblocks - 1) / mblocks;
+  s = std::min(s, 8);
+  s = std::min(s, std::max(1, kt_total / 4));
+  return std::max(1, std::min(s, kt_total));
+}
+
+}  // namespace
+
+svdq_status launch_act_quant(const ActArgs& a, cudaStream_t stream) {
+  const int mblocks = (a.M + 127) / 128;
+  const int kt_total = a.K / 64;
+  int splits = a.splits > 0 ? std::min(std::min(a.splits, 8), kt_total) : auto_splits(mblocks, kt_total);
+
+  CUtensorMap map_x;
+  svdq_status st = make_tmap_2d(&map_x, a.X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.K, a.M,
+                                static_cast<uint64_t>(a.K) * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != SVDQ_OK) return st;
+  CUtensorMap map_l1 = a.r_pad > 0 ? *a.map_l1 : map_x;
+
+  K1Params p;
+  p.M = a.M;
+  p.K = a.K;
+  p.r_pad = a.r_pad;
+  p.kt_total = kt_total;
+  p.splits = splits;
+  p.inv_lam = a.inv_lam;
+  p.xq = a.xq;
+  p.xsf = a.xsf;
+  p.T = a.T;
+  p.err = device_error_word();
+  p.wait_ns = wait_limit_ns();
+  p.stall = a.stall;
+  p.l1_tile = static_cast<uint32_t>(a.r_pad) * 128u;
+  uint32_t cols = 32;
+  while (cols < static_cast<uint32_t>(a.r_pad)) cols <<= 1;
+  p.tmem_cols = cols;
+  if (!p.err) return fail(SVDQ_ERR_CUDA, "device error word unavailable");
+
+  const size_t smem = 1024 + kStages * (kXTile + p.l1_tile) + sizeof(K1Shared);
+  static bool attr_set = false;
+  if (!attr_set) {
+    SVDQ_CUDA_TRY(cudaFuncSetAttribute(act_quant_lowrank_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
+    attr_set = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(mblocks, splits, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = splits;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  SVDQ_CUDA_TRY(cudaLaunchKernelEx(&cfg, act_quant_lowrank_kernel, map_x, map_l1, p));
+  return SVDQ_OK;
+}
+
+}  // namespace svdq

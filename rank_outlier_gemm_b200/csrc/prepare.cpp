@@ -1,0 +1,288 @@
+// Offline weight transform on the host, in float64.
+//
+// SVDQuant (paperlayer.ai summary of arXiv 2411.05007v4):
+//  * smoothing (§4.2; App. D, following SmoothQuant): per input channel j,
+//    lam_j = act_absmax_j^alpha / max_n |W_nj|^(1-alpha); lam_j = 1 when either
+//    maximum is 0.  The runtime multiplies activations by inv_lam = fp32(1/lam);
+//    the smoothed weight is W_hat = W diag(1/inv_lam).
+//  * low-rank split (§4.2): the top-r singular triplets of W_hat.  Computed by
+//    randomized subspace iteration with Rayleigh-Ritz (Halko, Martinsson and
+//    Tropp, "Finding structure with randomness", 2011, Alg. 4.4 + 5.1): a
+//    Gaussian start of r + p columns, q rounds of W_hat^T / W_hat products with
+//    re-orthonormalization, then the exact SVD of the small projected matrix
+//    through the eigen-decomposition of B B^T (cyclic Jacobi).
+//  * factors: L1 = U_r S_r (K x r), L2 = V_r^T (r x N); stored as
+//    L1' = bf16(diag(inv_lam) L1) and L2b = bf16(L2); the residual absorbs the
+//    factor rounding: R = W_hat - (diag(1/inv_lam) L1' L2b)^T.
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <functional>
+#include <random>
+#include <thread>
+#include <vector>
+
+#include "svdq_internal.h"
+
+namespace svdq {
+
+uint16_t f32_to_bf16_rne(float x) {
+  uint32_t u;
+  std::memcpy(&u, &x, 4);
+  if ((u & 0x7F800000u) == 0x7F800000u) return static_cast<uint16_t>(u >> 16);  // inf/nan
+  u += 0x7FFFu + ((u >> 16) & 1u);
+  return static_cast<uint16_t>(u >> 16);
+}
+
+float bf16_to_f32(uint16_t b) {
+  const uint32_t u = static_cast<uint32_t>(b) << 16;
+  float f;
+  std::memcpy(&f, &u, 4);
+  return f;
+}
+
+float weight_factor(const float* R, size_t n) {
+  double m = 0.0;
+  for (size_t i = 0; i < n; ++i) m = std::max(m, std::fabs(static_cast<double>(R[i])));
+  if (m == 0.0) return 1.0f;
+  int e = 0;
+  const double frac = std::frexp(m / (6.0 * 448.0), &e);  // m' = frac * 2^e, frac in [0.5, 1)
+  const int c = frac == 0.5 ? e - 1 : e;                  // ceil(log2(m'))
+  return static_cast<float>(std::ldexp(1.0, c));
+}
+
+namespace {
+
+void parallel_for(long n, const std::function<void(long, long)>& body) {
+  const long hw = std::max(1u, std::thread::hardware_concurrency());
+  const long nt = std::max(1L, std::min(hw, n / 4 + 1));
+  if (nt == 1) {
+    body(0, n);
+    return;
+  }
+  std::vector<std::thread> ts;
+  const long chunk = (n + nt - 1) / nt;
+  for (long t = 0; t < nt; ++t) {
+    const long b = t * chunk, e = std::min(n, b + chunk);
+    if (b < e) ts.emplace_back(body, b, e);
+  }
+  for (auto& t : ts) t.join();
+}
+
+// Y[N x l] = A[N x K] * X[K x l]   (all row-major)
+void mul_a_x(const std::vector<double>& A, int N, int K, const std::vector<double>& X, int l,
+             std::vector<double>& Y) {
+  Y.assign(static_cast<size_t>(N) * l, 0.0);
+  parallel_for(N, [&](long b, long e) {
+    std::vector<double> acc(l);
+    for (long n = b; n < e; ++n) {
+      std::fill(acc.begin(), acc.end(), 0.0);
+      const double* a = &A[static_cast<size_t>(n) * K];
+      for (int k = 0; k < K; ++k) {
+        const double w = a[k];
+        const double* x = &X[static_cast<size_t>(k) * l];
+        for (int j = 0; j < l; ++j) acc[j] += w * x[j];
+      }
+      std::copy(acc.begin(), acc.end(), &Y[static_cast<size_t>(n) * l]);
+    }
+  });
+}
+
+// Z[K x l] = A^T[K x N] * Q[N x l]
+void mul_at_q(const std::vector<double>& A, int N, int K, const std::vector<double>& Q, int l,
+              std::vector<double>& Z) {
+  Z.assign(static_cast<size_t>(K) * l, 0.0);
+  parallel_for(K, [&](long b, long e) {
+    for (int n = 0; n < N; ++n) {
+      const double* a = &A[static_cast<size_t>(n) * K];
+      const double* q = &Q[static_cast<size_t>(n) * l];
+      for (long k = b; k < e; ++k) {
+        const double w = a[k];
+        if (w == 0.0) continue;
+        double* z = &Z[static_cast<size_t>(k) * l];
+        for (int j = 0; j < l; ++j) z[j] += w * q[j];
+      }
+    }
+  });
+}
+
+// Orthonormalizes the l columns of a row-major [rows x l] matrix in place
+// (modified Gram-Schmidt, applied twice for stability).
+void orthonormalize(std::vector<double>& M, int rows, int l) {
+  std::vector<double> c(static_cast<size_t>(l) * rows);
+  for (int i = 0; i < rows; ++i)
+    for (int j = 0; j < l; ++j) c[static_cast<size_t>(j) * rows + i] = M[static_cast<size_t>(i) * l + j];
+  for (int pass = 0; pass < 2; ++pass) {
+    for (int j = 0; j < l; ++j) {
+      double* cj = &c[static_cast<size_t>(j) * rows];
+      for (int p = 0; p < j; ++p) {
+        const double* cp = &c[static_cast<size_t>(p) * rows];
+        double d = 0.0;
+        for (int i = 0; i < rows; ++i) d += cp[i] * cj[i];
+        for (int i = 0; i < rows; ++i) cj[i] -= d * cp[i];
+      }
+      double nrm = 0.0;
+      for (int i = 0; i < rows; ++i) nrm += cj[i] * cj[i];
+      nrm = std::sqrt(nrm);
+      const double inv = nrm > 0.0 ? 1.0 / nrm : 0.0;
+      for (int i = 0; i < rows; ++i) cj[i] *= inv;
+    }
+  }
+  for (int i = 0; i < rows; ++i)
+    for (int j = 0; j < l; ++j) M[static_cast<size_t>(i) * l + j] = c[static_cast<size_t>(j) * rows + i];
+}
+
+// Cyclic Jacobi eigen-decomposition of a symmetric [n x n] matrix G (row-major).
+// On return d holds the eigenvalues (descending) and E the matching
+// eigenvectors as columns.
+void jacobi_eigen(std::vector<double> G, int n, std::vector<double>& d, std::vector<double>& E) {
+  E.assign(static_cast<size_t>(n) * n, 0.0);
+  for (int i = 0; i < n; ++i) E[static_cast<size_t>(i) * n + i] = 1.0;
+  auto g = [&](int i, int j) -> double& { return G[static_cast<size_t>(i) * n + j]; };
+  for (int sweep = 0; sweep < 100; ++sweep) {
+    double off = 0.0, diag = 0.0;
+    for (int i = 0; i < n; ++i) {
+      diag += g(i, i) * g(i, i);
+      for (int j = i + 1; j < n; ++j) off += g(i, j) * g(i, j);
+    }
+    if (off <= 1e-30 * diag || off == 0.0) break;
+    for (int p = 0; p < n; ++p) {
+      for (int q = p + 1; q < n; ++q) {
+        const double apq = g(p, q);
+        if (std::fabs(apq) < 1e-300) continue;
+        const double theta = (g(q, q) - g(p, p)) / (2.0 * apq);
+        const double t = (theta >= 0 ? 1.0 : -1.0) / (std::fabs(theta) + std::sqrt(theta * theta + 1.0));
+        const double c = 1.0 / std::sqrt(t * t + 1.0), s = t * c;
+        for (int k = 0; k < n; ++k) {  // G <- J^T G J
+          const double gkp = g(k, p), gkq = g(k, q);
+          g(k, p) = c * gkp - s * gkq;
+          g(k, q) = s * gkp + c * gkq;
+        }
+        for (int k = 0; k < n; ++k) {
+          const double gpk = g(p, k), gqk = g(q, k);
+          g(p, k) = c * gpk - s * gqk;
+          g(q, k) = s * gpk + c * gqk;
+        }
+        for (int k = 0; k < n; ++k) {
+          double* e = &E[static_cast<size_t>(k) * n];
+          const double ekp = e[p], ekq = e[q];
+          e[p] = c * ekp - s * ekq;
+          e[q] = s * ekp + c * ekq;
+        }
+      }
+    }
+  }
+  std::vector<int> order(n);
+  for (int i = 0; i < n; ++i) order[i] = i;
+  std::sort(order.begin(), order.end(), [&](int a, int b) { return g(a, a) > g(b, b); });
+  d.resize(n);
+  std::vector<double> Es(static_cast<size_t>(n) * n);
+  for (int j = 0; j < n; ++j) {
+    d[j] = g(order[j], order[j]);
+    for (int k = 0; k < n; ++k) Es[static_cast<size_t>(k) * n + j] = E[static_cast<size_t>(k) * n + order[j]];
+  }
+  E.swap(Es);
+}
+
+}  // namespace
+
+svdq_status host_prepare_split(const uint16_t* W_bf16, const float* act_absmax, int N, int K,
+                               const svdq_prepare_opts& o, HostSplit* out) {
+  const int r = o.rank;
+  // ---- smoothing
+  std::vector<double> wmax(K, 0.0);
+  for (int n = 0; n < N; ++n)
+    for (int k = 0; k < K; ++k)
+      wmax[k] = std::max(wmax[k], std::fabs(static_cast<double>(bf16_to_f32(W_bf16[static_cast<size_t>(n) * K + k]))));
+  out->inv_lam.resize(K);
+  for (int k = 0; k < K; ++k) {
+    const double ax = act_absmax[k];
+    double lam = 1.0;
+    if (ax > 0.0 && wmax[k] > 0.0) lam = std::pow(ax, static_cast<double>(o.alpha)) / std::pow(wmax[k], 1.0 - o.alpha);
+    const float lam32 = static_cast<float>(lam);
+    out->inv_lam[k] = static_cast<float>(1.0 / static_cast<double>(lam32));
+  }
+  std::vector<double> Wh(static_cast<size_t>(N) * K);
+  parallel_for(N, [&](long b, long e) {
+    for (long n = b; n < e; ++n)
+      for (int k = 0; k < K; ++k)
+        Wh[static_cast<size_t>(n) * K + k] =
+            static_cast<double>(bf16_to_f32(W_bf16[static_cast<size_t>(n) * K + k])) /
+            static_cast<double>(out->inv_lam[k]);
+  });
+
+  out->L1p.assign(static_cast<size_t>(K) * r, 0);
+  out->L2.assign(static_cast<size_t>(r) * N, 0);
+  std::vector<double> L1s(static_cast<size_t>(K) * r, 0.0), L2d(static_cast<size_t>(r) * N, 0.0);
+  if (r > 0) {
+    // ---- randomized subspace iteration
+    const int l = std::min(r + std::max(0, o.oversample), std::min(N, K));
+    std::mt19937_64 gen(o.seed);
+    std::normal_distribution<double> nd(0.0, 1.0);
+    std::vector<double> Om(static_cast<size_t>(K) * l);
+    for (auto& v : Om) v = nd(gen);
+    std::vector<double> Y, Z, Q;
+    mul_a_x(Wh, N, K, Om, l, Y);
+    orthonormalize(Y, N, l);
+    for (int it = 0; it < std::max(0, o.power_iters); ++it) {
+      mul_at_q(Wh, N, K, Y, l, Z);
+      orthonormalize(Z, K, l);
+      mul_a_x(Wh, N, K, Z, l, Y);
+      orthonormalize(Y, N, l);
+    }
+    Q.swap(Y);                       // N x l, orthonormal columns
+    mul_at_q(Wh, N, K, Q, l, Z);     // Z = W_hat^T Q = B^T  (K x l)
+    // ---- Rayleigh-Ritz: eigen-decomposition of B B^T = Z^T Z (l x l)
+    std::vector<double> G(static_cast<size_t>(l) * l, 0.0);
+    for (int a = 0; a < l; ++a)
+      for (int b = a; b < l; ++b) {
+        double s = 0.0;
+        for (int k = 0; k < K; ++k) s += Z[static_cast<size_t>(k) * l + a] * Z[static_cast<size_t>(k) * l + b];
+        G[static_cast<size_t>(a) * l + b] = G[static_cast<size_t>(b) * l + a] = s;
+      }
+    std::vector<double> d, E;
+    jacobi_eigen(G, l, d, E);
+    // L2 = (Q E_r)^T, L1 = B^T E_r = Z E_r
+    for (int i = 0; i < r; ++i) {
+      for (int n = 0; n < N; ++n) {
+        double s = 0.0;
+        for (int a = 0; a < l; ++a) s += Q[static_cast<size_t>(n) * l + a] * E[static_cast<size_t>(a) * l + i];
+        L2d[static_cast<size_t>(i) * N + n] = s;
+      }
+      for (int k = 0; k < K; ++k) {
+        double s = 0.0;
+        for (int a = 0; a < l; ++a) s += Z[static_cast<size_t>(k) * l + a] * E[static_cast<size_t>(a) * l + i];
+        L1s[static_cast<size_t>(k) * r + i] = s;
+      }
+    }
+    // ---- 16-bit factors; the residual uses them as the runtime does
+    for (int k = 0; k < K; ++k)
+      for (int i = 0; i < r; ++i) {
+        const double v = static_cast<double>(out->inv_lam[k]) * L1s[static_cast<size_t>(k) * r + i];
+        const uint16_t b = f32_to_bf16_rne(static_cast<float>(v));
+        out->L1p[static_cast<size_t>(k) * r + i] = b;
+        L1s[static_cast<size_t>(k) * r + i] = static_cast<double>(bf16_to_f32(b)) / static_cast<double>(out->inv_lam[k]);
+      }
+    for (size_t i = 0; i < L2d.size(); ++i) {
+      const uint16_t b = f32_to_bf16_rne(static_cast<float>(L2d[i]));
+      out->L2[i] = b;
+      L2d[i] = bf16_to_f32(b);
+    }
+  }
+  out->R.resize(static_cast<size_t>(N) * K);
+  parallel_for(N, [&](long b, long e) {
+    std::vector<double> l2n(std::max(r, 1));
+    for (long n = b; n < e; ++n) {
+      for (int i = 0; i < r; ++i) l2n[i] = L2d[static_cast<size_t>(i) * N + n];
+      for (int k = 0; k < K; ++k) {
+        double low = 0.0;
+        const double* l1 = &L1s[static_cast<size_t>(k) * r];
+        for (int i = 0; i < r; ++i) low += l1[i] * l2n[i];
+        out->R[static_cast<size_t>(n) * K + k] = static_cast<float>(Wh[static_cast<size_t>(n) * K + k] - low);
+      }
+    }
+  });
+  return SVDQ_OK;
+}
+
+}  // namespace svdq

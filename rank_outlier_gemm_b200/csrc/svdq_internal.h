@@ -1,0 +1,114 @@
+// Internal declarations shared by the library's host code and kernel launchers.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+#include <vector>
+
+#include "svdq.h"
+
+namespace svdq {
+
+// Records a failure message for svdq_last_error() and returns `s`.
+svdq_status fail(svdq_status s, const char* fmt, ...);
+// Maps a CUDA runtime error to SVDQ_ERR_CUDA with a message.
+svdq_status cuda_fail(cudaError_t e, const char* what);
+
+#define SVDQ_CUDA_TRY(expr)                                 \
+  do {                                                      \
+    cudaError_t _e = (expr);                                \
+    if (_e != cudaSuccess) return ::svdq::cuda_fail(_e, #expr); \
+  } while (0)
+
+// Device error word of the current device (lazily allocated, zeroed).
+int* device_error_word();
+uint64_t wait_limit_ns();
+// SVDQ_OK if the current device is sm_100, else SVDQ_ERR_UNSUPPORTED_DEVICE.
+svdq_status check_device();
+
+// 2-D tiled tensor map over a row-major [outer, inner] array.
+svdq_status make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
+                         uint64_t inner, uint64_t outer, uint64_t row_bytes, uint32_t box_inner,
+                         uint32_t box_outer, CUtensorMapSwizzle swizzle);
+
+inline int round_up(int x, int m) { return (x + m - 1) / m * m; }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ------------------------------------------------------------- kernels
+struct ActArgs {
+  int M, K, r_pad;
+  const void* X;            // device bf16 [M, K]
+  const CUtensorMap* map_l1;  // L1'^T [r_pad, K] bf16 (ignored when r_pad == 0)
+  const float* inv_lam;     // device [K]
+  uint8_t* xq;
+  uint8_t* xsf;
+  uint16_t* T;              // device [M, 2 r_pad] bf16 (hi/lo chunks)
+  int stall;                // test hook: a wait that never completes
+  int splits;               // K-splits per 128-row block (0 = automatic)
+};
+svdq_status launch_act_quant(const ActArgs& a, cudaStream_t stream);
+
+struct GemmArgs {
+  int M, N, K, r_pad;
+  const void* xq;           // device [M, K/2]
+  const void* xsf;          // device act scales (atom layout)
+  const void* T;            // device [M, 2 r_pad] bf16
+  const CUtensorMap* map_wq_256;  // weight codes, box rows 256
+  const CUtensorMap* map_wq_128;  // weight codes, box rows 128
+  const CUtensorMap* map_l2_256;  // L2^T/alpha_w [N, r_pad] bf16, box rows 256
+  const CUtensorMap* map_l2_128;
+  const uint8_t* wsf;       // device weight scales (atom layout)
+  const float* bias;        // device [N]
+  float alpha_w;
+  void* Y;                  // device bf16 [M, N]
+  int force_bn;             // 0 = automatic, else 128 or 256
+};
+svdq_status launch_gemm_w4a4(const GemmArgs& a, cudaStream_t stream);
+
+// NVFP4 codes + atom-layout scales of a device fp32 [rows, K] matrix.
+svdq_status launch_weight_codec(const float* d_src, int rows, int K, uint8_t* codes, uint8_t* sf,
+                                cudaStream_t stream);
+
+// ------------------------------------------------------------- host math
+struct HostSplit {
+  std::vector<float> inv_lam;      // [K]
+  std::vector<uint16_t> L1p;       // [K, r] bf16
+  std::vector<uint16_t> L2;        // [r, N] bf16
+  std::vector<float> R;            // [N, K]
+};
+// Smoothing + randomized SVD split + residual on the host (float64 math).
+svdq_status host_prepare_split(const uint16_t* W_bf16, const float* act_absmax, int N, int K,
+                               const svdq_prepare_opts& opts, HostSplit* out);
+uint16_t f32_to_bf16_rne(float x);
+float bf16_to_f32(uint16_t b);
+float weight_factor(const float* R, size_t n);
+
+}  // namespace svdq
+
+// The opaque handle.
+struct svdq_weights {
+  int device = 0;
+  int N = 0, K = 0;
+  int rank = 0;       // SVD rank + LoRA ranks
+  int r_pad = 0;      // rank rounded up to 16
+  float alpha_w = 1.0f;
+  uint8_t* d_wq = nullptr;       // [N, K/2]
+  uint8_t* d_wsf = nullptr;      // [ceil(N/128)*128, K/16] atom layout
+  float* d_inv_lam = nullptr;    // [K]
+  uint16_t* d_L1t = nullptr;     // [r_pad, K] bf16 = L1'^T
+  uint16_t* d_L2t = nullptr;     // [N, r_pad] bf16 = L2^T / alpha_w
+  float* d_bias = nullptr;       // [N]
+  // host copies (export, LoRA growth)
+  std::vector<float> inv_lam;
+  std::vector<uint16_t> L1p;     // [K, rank]
+  std::vector<uint16_t> L2;      // [rank, N]
+  std::vector<float> bias;
+  std::vector<float> residual;   // [N, K] R / alpha_w (only if kept)
+  // tensor maps over the weight-side buffers
+  CUtensorMap map_l1{};
+  CUtensorMap map_wq_256{}, map_wq_128{};
+  CUtensorMap map_l2_256{}, map_l2_128{};
+};

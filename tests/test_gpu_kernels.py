@@ -1,0 +1,190 @@
+"""GPU parity of the two kernels against the CPU oracle, through the C ABI.
+
+Codes and scales must match bit for bit; Y must be within the layer
+tolerance (relative Frobenius 2e-3, per element 1e-2 * max(1, |ref|)); on
+inputs that already lie on the FP4 grid Y must equal bf16(X W^T) exactly."""
+
+import functools
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import codec as OC
+from oracle import formats as OF
+from oracle import svdquant as OS
+from synth import config_cases, f32_to_bf16_bits, make_fp4_grid_inputs, make_layer_inputs
+from tests import gpu_common as G
+
+pytestmark = pytest.mark.gpu
+
+
+@functools.lru_cache(maxsize=None)
+def _case_prep(label: str, M: int):
+    cfg, name = label.split("/")
+    case = [c for c in config_cases(cfg) if c.name == name][0]
+    t = make_layer_inputs(case, M=M)
+    prep = OS.prepare(t.W, t.act_absmax, t.bias, case.rank)
+    return t, prep
+
+
+def _rank0_prep(W, inv_lam, bias=None):
+    K = W.shape[1]
+    W_hat = OS.smooth_weight(W, inv_lam)
+    return OS.prepare_from_factors(W_hat, inv_lam, np.zeros((K, 0)), np.zeros((0, W.shape[0])), bias)
+
+
+@pytest.mark.parametrize("M,K", [(64, 256), (1, 64), (200, 640), (333, 3072), (128, 1152)])
+def test_activation_codes_bitexact(M, K):
+    rng = np.random.default_rng(M * 7 + K)
+    X = rng.normal(0, 1, (M, K)).astype(np.float32)
+    X[:, rng.choice(K, 3, replace=False)] *= 50
+    X[0, :32] = 0.0                       # an all-zero group
+    X[-1, 16:32] = 1e-7                   # scale rounds to zero
+    X[-1, 32:48] = -1e-3                  # E4M3 subnormal scale, negatives
+    X[min(1, M - 1), 48:64] = 3e4         # large values
+    Xb = f32_to_bf16_bits(X)
+    Xf = OF.bf16_bits_to_f64(Xb).astype(np.float32)
+    inv_lam = np.exp2(rng.uniform(-3, 3, K)).astype(np.float32)
+    W = rng.normal(0, 0.02, (64, K)).astype(np.float32)
+    w = G.weights_from_oracle(_rank0_prep(W, inv_lam))
+    _, xq, xsf, T = G.run_act(w, Xb)
+    assert T is None
+    G.check_codes(xq, xsf, Xf, inv_lam)
+
+
+def test_weight_codes_and_factor_bitexact():
+    t, prep = _case_prep("pixart/attn_qkv_out", 128)
+    w = G.weights_from_oracle(prep)
+    ex = G.lib().svdq_weights_export(w, residual=True)
+    assert ex["alpha_w"] == prep.alpha_w
+    np.testing.assert_array_equal(ex["residual"], prep.Rp)
+    np.testing.assert_array_equal(ex["codes"], OC.pack_codes(prep.w_codes))
+    np.testing.assert_array_equal(ex["sf"], OC.scales_to_atoms(prep.w_scales))
+
+
+@pytest.mark.parametrize("M,K,N", [(128, 256, 256), (64, 256, 48), (300, 640, 400), (77, 1280, 512)])
+def test_exact_product_on_fp4_grid(M, K, N):
+    Xb, X, Wb, W = make_fp4_grid_inputs(M, K, N, seed=M + K + N)
+    w = G.weights_from_oracle(_rank0_prep(W, np.ones(K, np.float32)))
+    Y, (xq, xsf, _) = G.run_layer(w, Xb)
+    G.check_codes(xq, xsf, X, np.ones(K, np.float32))
+    exact = X.astype(np.float64) @ W.astype(np.float64).T
+    np.testing.assert_array_equal(Y, OF.round_bf16(exact))
+
+
+def test_tiny_layer():
+    t, prep = _case_prep("tiny/layer", 64)
+    w = G.weights_from_oracle(prep)
+    Y, (xq, xsf, T) = G.run_layer(w, t.X_bits)
+    G.check_codes(xq, xsf, t.X, prep.inv_lam)
+    G.check_T(T, t.X, prep)
+    G.check_Y(Y, OS.linear(prep, t.X))
+
+
+def test_rank0_plain_w4a4_layer():
+    t, _ = _case_prep("tiny/layer", 64)
+    K = t.case.K
+    prep = OS.prepare_from_factors(t.W, np.ones(K, np.float32), np.zeros((K, 0)), np.zeros((0, t.case.N)),
+                                   t.bias)
+    w = G.weights_from_oracle(prep)
+    Y, _ = G.run_layer(w, t.X_bits)
+    G.check_Y(Y, OS.linear(prep, t.X))
+
+
+ALL_LAYERS = [c.label for cfg in ["pixart", "flux", "sdxl", "small_m_lora"] for c in config_cases(cfg)]
+
+
+@pytest.mark.parametrize("label", ALL_LAYERS)
+def test_config_layer_reduced_M(label):
+    """Every configured layer at full K, N with 300 tokens (3 row tiles, ragged)."""
+    cfg, name = label.split("/")
+    case = [c for c in config_cases(cfg) if c.name == name][0]
+    M = min(case.M, 300)
+    t, prep = _case_prep(label, M)
+    w = G.weights_from_oracle(prep)
+    ref_prep = prep
+    if case.lora_rank:
+        G.lib().svdq_attach_lora(w, t.lora_A_bits, t.lora_B_bits, t.lora_scale)
+        ref_prep = OS.attach_lora(prep, t.lora_A, t.lora_B, t.lora_scale)
+    Y, (xq, xsf, T) = G.run_layer(w, t.X_bits)
+    G.check_codes(xq, xsf, t.X, prep.inv_lam)
+    G.check_T(T, t.X, ref_prep)
+    G.check_Y(Y, OS.linear(ref_prep, t.X))
+
+
+def test_lora_attach_keeps_codes():
+    t, prep = _case_prep("small_m_lora/M16_N3072", 16)
+    w = G.weights_from_oracle(prep)
+    before = G.lib().svdq_weights_export(w)
+    G.lib().svdq_attach_lora(w, t.lora_A_bits, t.lora_B_bits, 0.5)
+    after = G.lib().svdq_weights_export(w)
+    for k in ("codes", "sf", "inv_lam", "bias"):
+        np.testing.assert_array_equal(before[k], after[k])
+    assert after["rank"] == before["rank"] + 16 and after["alpha_w"] == before["alpha_w"]
+    np.testing.assert_array_equal(after["L1p"][:, 32:], t.lora_A_bits)
+    ref = OS.attach_lora(prep, t.lora_A, t.lora_B, 0.5)
+    Y, _ = G.run_layer(w, t.X_bits)
+    G.check_Y(Y, OS.linear(ref, t.X))
+
+
+def test_forward_entry_points_agree():
+    L = G.lib()
+    t, prep = _case_prep("pixart/mlp_up", 300)
+    w = G.weights_from_oracle(prep)
+    Y2, _ = G.run_layer(w, t.X_bits)
+    M = t.X_bits.shape[0]
+    X = G.to_dev_bf16(t.X_bits)
+    Y = torch.empty((M, w.info["N"]), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(L.svdq_forward_workspace_bytes(w, M), dtype=torch.uint8, device="cuda")
+    L.svdq_forward(w, X, Y, ws)
+    assert L.svdq_check_device_errors() == 0
+    np.testing.assert_array_equal(Y.float().cpu().numpy(), Y2)
+    Xh = torch.from_numpy(t.X_bits.view(np.int16).copy()).view(torch.bfloat16).pin_memory()
+    Yh = torch.empty((M, w.info["N"]), dtype=torch.bfloat16).pin_memory()
+    wsh = torch.empty(L.svdq_forward_host_workspace_bytes(w, M), dtype=torch.uint8, device="cuda")
+    L.svdq_forward_host(w, Xh, Yh, wsh)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(Yh.float().numpy(), Y2)
+
+
+def test_library_prepare_invariants():
+    """The library's own host SVD split: inv_lam as the oracle's, L1 L2 + R
+    reconstructs W_hat, and the split is near the Eckart-Young optimum."""
+    L = G.lib()
+    t, prep = _case_prep("tiny/layer", 64)
+    w = L.svdq_prepare_weights(t.W_bits, t.act_absmax, t.bias_bits, rank=16, keep_residual=True)
+    ex = L.svdq_weights_export(w, residual=True)
+    np.testing.assert_allclose(ex["inv_lam"], prep.inv_lam, rtol=1.2e-7, atol=0)
+    W_hat = OS.smooth_weight(t.W, ex["inv_lam"])
+    L1p = OF.bf16_bits_to_f64(ex["L1p"])
+    L2 = OF.bf16_bits_to_f64(ex["L2"])
+    low = ((L1p / ex["inv_lam"].astype(np.float64)[:, None]) @ L2).T
+    recon = low + ex["residual"].astype(np.float64) * ex["alpha_w"]
+    assert np.linalg.norm(recon - W_hat) / np.linalg.norm(W_hat) < 1e-6
+    opt = np.sum(prep.sigma[16:] ** 2)
+    assert np.linalg.norm(W_hat - low) ** 2 <= 1.02 * opt + 1e-3 * np.sum(prep.sigma ** 2)
+    np.testing.assert_allclose(np.linalg.svd(low, compute_uv=False)[:16], prep.sigma[:16], rtol=2e-2)
+    # its layer output is as accurate as the oracle's own split
+    Y, _ = G.run_layer(w, t.X_bits)
+    exact = t.X.astype(np.float64) @ t.W.astype(np.float64).T + t.bias
+    e_lib = np.linalg.norm(Y - exact) / np.linalg.norm(exact)
+    e_orc = np.linalg.norm(OS.linear(prep, t.X) - exact) / np.linalg.norm(exact)
+    assert e_lib < 1.5 * e_orc + 1e-3
+
+
+def test_bounded_wait_reports_timeout():
+    L = G.lib()
+    t, prep = _case_prep("tiny/layer", 64)
+    w = G.weights_from_oracle(prep)
+    X = G.to_dev_bf16(t.X_bits)
+    xq, xsf, T = L.act_buffers(w, 64)
+    L.svdq_set_wait_limit_ns(2_000_000)
+    try:
+        L.svdq_debug_launch_stalled_act(w, X, xq, xsf, T)
+        assert L.svdq_check_device_errors() == 5          # SVDQ_ERR_TIMEOUT
+    finally:
+        L.svdq_set_wait_limit_ns(2_000_000_000)
+    # the context is still usable and the error word was cleared
+    Y, _ = G.run_layer(w, t.X_bits)
+    G.check_Y(Y, OS.linear(prep, t.X))
