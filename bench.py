@@ -1,0 +1,381 @@
+#!/usr/bin/env python3
+"""Benchmark of the fused SVDQuant W4A4 + low-rank linear layer on B200.
+
+One step = the hot path over one FLUX.1 double-block's linears (M = 4608
+tokens: attn-out 3072->3072, fused qkv 3072->9216, MLP-up 3072->12288,
+MLP-down 12288->3072; rank 32), each layer = activation kernel + GEMM kernel.
+The metric is whole-job FP4 GEMM throughput 2*M*N*K / time (TFLOP/s), plus
+us per layer.  With torchrun every rank runs its own replica of the step on
+its own batch (weak scaling; the layer needs no collective), and the time is
+the max over ranks.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+``--impl reference`` times the CPU oracle on a bounded row sample of the
+same workload on the host cores.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synth import config_cases, make_layer_inputs  # noqa: E402
+
+METRIC = "fused W4A4+low-rank linear TFLOPS & % of FP4 roofline; us/layer on FLUX shapes"
+WORKLOAD = "FLUX.1 double-block linears (attn_out, qkv, mlp_up, mlp_down), M=4608, rank 32, NVFP4 g16"
+NOMINAL_FP4_OVER_BF16 = 4.0      # dense FP4 : dense BF16 tensor rate (9 : 2.25 PFLOP/s)
+FALLBACK_BF16_SUSTAINED = 1400.0
+FALLBACK_BF16_BURST = 1590.0
+FALLBACK_HBM = 6650.0
+
+SMI_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return {"bf16": d["bf16_tflops"], "bf16_sustained": d["bf16_tflops_sustained"],
+                "hbm": d["hbm_gbs"], "source": "measured"}
+    except Exception:
+        return {"bf16": FALLBACK_BF16_BURST, "bf16_sustained": FALLBACK_BF16_SUSTAINED,
+                "hbm": FALLBACK_HBM, "source": "fallback"}
+
+
+LAYER_FILTER = None
+
+
+def flux_cases():
+    cs = config_cases("flux")
+    if LAYER_FILTER:
+        cs = [c for c in cs if c.name in LAYER_FILTER]
+    return cs
+
+
+def layer_bytes(c) -> float:
+    """Minimum HBM bytes of one layer: X read, weight codes+scales, Y write."""
+    return 2 * c.M * c.K + c.N * c.K * (0.5 + 1 / 16) + 2 * c.M * c.N
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    def __init__(self, gpu_index: int):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.p = None
+        self.gpu = gpu_index
+
+    def __enter__(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={SMI_FIELDS}",
+                                       "--format=csv,noheader,nounits", "-lms", "100"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+        time.sleep(0.15)
+        return self
+
+    def __exit__(self, *a):
+        if self.p:
+            time.sleep(0.15)
+            self.p.terminate()
+            try:
+                self.p.wait(timeout=5)
+            except Exception:
+                self.p.kill()
+
+    def summary(self):
+        try:
+            rows = [l.strip().split(",") for l in open(self.f.name) if l.strip()]
+            os.unlink(self.f.name)
+        except Exception:
+            return None
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if len(r) >= 9]
+        mx = [float(r[2]) for r in rows if len(r) >= 9]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows if len(r) >= 9 for i in range(4)
+                          if r[5 + i].strip().lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ ours
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=torch.device("cuda", local))
+    import rank_outlier_gemm_b200 as L
+
+    dev = torch.device("cuda", local)
+    cases = flux_cases()
+    layers = []
+    for c in cases:
+        t = make_layer_inputs(c)
+        w = L.svdq_prepare_weights(t.W_bits, t.act_absmax, t.bias_bits, rank=c.rank)
+        w0 = L.svdq_prepare_weights(t.W_bits, t.act_absmax, t.bias_bits, rank=0) if args.extras else None
+        X = torch.from_numpy(t.X_bits.view(np.int16).copy()).view(torch.bfloat16).to(dev)
+        bufs = L.act_buffers(w, c.M, dev)
+        Y = torch.empty((c.M, c.N), dtype=torch.bfloat16, device=dev)
+        layers.append(dict(case=c, w=w, w0=w0, X=X, bufs=bufs, Y=Y, X_bits=t.X_bits))
+    stream = torch.cuda.current_stream()
+
+    def step(evs=None):
+        for i, l in enumerate(layers):
+            xq, xsf, T = l["bufs"]
+            if evs is not None:
+                evs[i][0].record(stream)
+            L.svdq_quantize_act_lowrank_down(l["w"], l["X"], xq, xsf, T)
+            if evs is not None:
+                evs[i][1].record(stream)
+            L.svdq_linear_w4a4(l["w"], xq, xsf, T, l["case"].M, l["Y"])
+            if evs is not None:
+                evs[i][2].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step()
+    assert L.svdq_check_device_errors() == 0
+    nl = len(layers)
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(nl)]
+           for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    with ClockSampler(local) as cs:
+        t0.record(stream)
+        for s in range(args.steps):
+            step(evs[s])
+        t1.record(stream)
+        barrier()
+    assert L.svdq_check_device_errors() == 0
+    ms = max_over_ranks(t0.elapsed_time(t1))
+    ms_step = ms / args.steps
+    k1 = [statistics.mean(evs[s][i][0].elapsed_time(evs[s][i][1]) for s in range(args.steps)) for i in range(nl)]
+    k2 = [statistics.mean(evs[s][i][1].elapsed_time(evs[s][i][2]) for s in range(args.steps)) for i in range(nl)]
+    flops_step = sum(l["case"].flops for l in layers)
+    value = world * flops_step / (ms_step * 1e-3) / 1e12
+
+    pk = peaks()
+    fp4_peak = pk["bf16_sustained"] * NOMINAL_FP4_OVER_BF16
+    k2_flops = flops_step
+    k2_ms = sum(k2)
+    achieved = k2_flops / (k2_ms * 1e-3) / 1e12
+    roof_us = {l["case"].name: max(l["case"].flops / (fp4_peak * 1e12), layer_bytes(l["case"]) / (pk["hbm"] * 1e9)) * 1e6
+               for l in layers}
+
+    # low-rank overhead: the same kernels at rank 0 (extras)
+    overhead = None
+    if args.extras:
+        def step0():
+            for l in layers:
+                xq, xsf, _ = l["bufs"]
+                L.svdq_quantize_act_lowrank_down(l["w0"], l["X"], xq, xsf, None)
+                L.svdq_linear_w4a4(l["w0"], xq, xsf, None, l["case"].M, l["Y"])
+        n0 = max(10, args.steps // 4)
+        for _ in range(3):
+            step0()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record(stream)
+        for _ in range(n0):
+            step0()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms0 = a.elapsed_time(b) / n0
+        overhead = ms_step / ms0 - 1.0
+
+    # end to end through the public host-buffer call: H2D of X, both kernels, D2H of Y
+    e2e = None
+    if args.e2e_steps > 0:
+        host = []
+        for l in layers:
+            c = l["case"]
+            Xh = torch.from_numpy(l["X_bits"].view(np.int16).copy()).view(torch.bfloat16).pin_memory()
+            Yh = torch.empty((c.M, c.N), dtype=torch.bfloat16).pin_memory()
+            ws = torch.empty(L.svdq_forward_host_workspace_bytes(l["w"], c.M), dtype=torch.uint8, device=dev)
+            host.append((Xh, Yh, ws))
+
+        def step_e2e():
+            for l, (Xh, Yh, ws) in zip(layers, host):
+                L.svdq_forward_host(l["w"], Xh, Yh, ws)
+
+        step_e2e()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            step_e2e()
+        b.record(stream)
+        barrier()
+        ems = max_over_ranks(a.elapsed_time(b)) / args.e2e_steps
+        h2d = sum(l["case"].M * l["case"].K * 2 for l in layers)
+        d2h = sum(l["case"].M * l["case"].N * 2 for l in layers)
+        e2e = {"value": world * flops_step / (ems * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ems,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
+
+    if rank == 0:
+        out = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic (seeded; FLUX.1 shapes, random weights)",
+            "config": {"workload": WORKLOAD, "M": cases[0].M, "layers": [[c.K, c.N] for c in cases],
+                       "rank": cases[0].rank, "parallelism": f"replicas x{world}",
+                       "l2": "step footprint ~0.5 GB > 126 MB L2; no flush"},
+            "us_per_layer": {l["case"].name: 1e3 * (k1[i] + k2[i]) for i, l in enumerate(layers)},
+            "us_act_kernel": {l["case"].name: 1e3 * k1[i] for i, l in enumerate(layers)},
+            "us_gemm_kernel": {l["case"].name: 1e3 * k2[i] for i, l in enumerate(layers)},
+            "roofline_us_per_layer": roof_us,
+            "frac_of_layer_roofline": sum(roof_us.values()) / (1e3 * (sum(k1) + sum(k2))),
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
+                         "frac": achieved / fp4_peak, "traffic": None,
+                         "kernel": "gemm_w4a4_kernel", "peak_source":
+                         f"{pk['source']} bf16 sustained {pk['bf16_sustained']} x {NOMINAL_FP4_OVER_BF16} (nominal FP4:BF16)",
+                         "frac_of_datasheet_9pf": achieved / 9000.0},
+            "lowrank_overhead_vs_rank0": overhead,
+            "gpu_launches": 2 * nl * args.steps,
+            "e2e": e2e,
+        }
+        cl = cs.summary()
+        if cl:
+            out["clocks"] = cl
+        if args.cpu_baseline and world == 1:
+            out["cpu_baseline"] = cpu_baseline(args.cpu_rows, reps=1)
+        print(json.dumps(out))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------ oracle
+def _oracle_layers():
+    from oracle import svdquant as OS
+    preps = []
+    for c in flux_cases():
+        t = make_layer_inputs(c)
+        preps.append((c, t, OS.prepare(t.W, t.act_absmax, t.bias, c.rank)))
+    return preps
+
+
+def cpu_baseline(rows: int, reps: int = 1, preps=None):
+    """The oracle's runtime step (activation codec, fp64 dequantized GEMM,
+    low-rank branch) on `rows` rows of every layer; weight preparation untimed."""
+    from oracle import svdquant as OS
+    preps = preps or _oracle_layers()
+    sample = np.arange(rows)
+    t = time.perf_counter()
+    for _ in range(reps):
+        for c, inp, prep in preps:
+            OS.linear(prep, inp.X, rows=sample)
+    dt = (time.perf_counter() - t) / reps
+    flops = sum(2 * rows * c.N * c.K for c, _, _ in preps)
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": _threads(), "kind": "oracle",
+            "sample": f"first {rows} of 4608 rows of each FLUX layer per step (weights full size)",
+            "seconds_per_step": dt}
+
+
+def _threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args):
+    """The oracle as the reference arm: each step computes a bounded sample of
+    the step's outputs (args.ref_rows rows x args.ref_cols output columns of
+    every layer) on the host cores; flops count only the sampled outputs."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from oracle import svdquant as OS
+    preps = _oracle_layers()
+    rows = np.arange(args.ref_rows)
+
+    def one_step(s):
+        for c, inp, prep in preps:
+            cols = (np.arange(args.ref_cols) * 7919 + s * 131) % c.N
+            OS.linear(prep, inp.X, rows=rows, cols=cols)
+
+    for s in range(args.warmup):
+        one_step(s)
+    t = time.perf_counter()
+    for s in range(args.steps):
+        one_step(s)
+    dt = (time.perf_counter() - t) / args.steps
+    flops = sum(2 * args.ref_rows * args.ref_cols * c.K for c, _, _ in preps)
+    v = flops / dt / 1e12
+    sample = (f"{args.ref_rows} rows x {args.ref_cols} output columns of each of the 4 FLUX layers "
+              f"per step (weights prepared untimed)")
+    out = {"metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded; FLUX.1 shapes, random weights)",
+           "config": {"workload": WORKLOAD, "M": 4608, "layers": [[c.K, c.N] for c, _, _ in preps],
+                      "rank": 32, "parallelism": "host cores"},
+           "impl": "reference",
+           "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": _threads(), "kind": "oracle",
+                            "sample": sample},
+           "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+           "gpu_launches": 0}
+    print(json.dumps(out))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-rows", type=int, default=16)
+    ap.add_argument("--ref-rows", type=int, default=2)
+    ap.add_argument("--ref-cols", type=int, default=64)
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--no-extras", dest="extras", action="store_false")
+    ap.add_argument("--layers", default="", help="comma-separated subset of the FLUX layers (profiling)")
+    args = ap.parse_args()
+    global LAYER_FILTER
+    LAYER_FILTER = [x for x in args.layers.split(",") if x] or None
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -153,15 +153,17 @@ def lowrank_down(X, prep: Prepared) -> np.ndarray:
     return np.asarray(X, np.float64) @ prep.L1p
 
 
-def linear(prep: Prepared, X, rows=None) -> np.ndarray:
-    """Y in float64 for all rows of X, or for the listed row indices."""
+def linear(prep: Prepared, X, rows=None, cols=None) -> np.ndarray:
+    """Y in float64 for all rows of X, or for the listed row indices and/or
+    output columns (the same arithmetic restricted to those outputs)."""
     X = np.asarray(X, np.float32)
     if rows is not None:
         X = X[np.asarray(rows)]
+    c = slice(None) if cols is None else np.asarray(cols)
     xc, xs = quantize_activations(X, prep.inv_lam)
-    main = dequantize_groups(xc, xs) @ dequantize_groups(prep.w_codes, prep.w_scales).T
+    main = dequantize_groups(xc, xs) @ dequantize_groups(prep.w_codes[c], prep.w_scales[c]).T
     L2 = prep.L2b if prep.lora_B_exact is None else prep.lora_B_exact
-    return prep.alpha_w * main + lowrank_down(X, prep) @ L2 + prep.bias[None, :]
+    return prep.alpha_w * main + lowrank_down(X, prep) @ L2[:, c] + prep.bias[None, c]
 
 
 def attach_lora(prep: Prepared, A, B, scale: float = 1.0) -> Prepared:
