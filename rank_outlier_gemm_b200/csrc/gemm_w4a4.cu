@@ -2,18 +2,24 @@
 // the same tensor-memory accumulator.
 //
 // SVDQuant §4.3 (Nunchaku, Fig. 6): the up-projection is fused into the 4-bit
-// computation kernel so the output tile is produced once.  Per 128 x BN tile:
-//   warp 0     producer: TMA loads of activation codes [128 x 256 FP4] and
-//              weight codes [BN x 256 FP4] (128-byte swizzled rows) plus 1-D
-//              bulk copies of the matching 512-byte scale atoms; then the
-//              low-rank slab: T (hi/lo bf16, 128-byte rows) and L2^T/alpha_w
-//              (64-byte rows)
-//   warp 1     MMA issuer: tcgen05.cp of the scale atoms into TMEM (two
-//              alternating buffers), tcgen05.mma kind::mxf4nvf4 block16
-//              (M=128, N=BN, K=64) per 64-element K block, then tcgen05.mma
-//              kind::f16 (K=16) for T_hi L2 and T_lo L2 into the same accumulator
-//   warps 2-5  epilogue: tcgen05.ld of the fp32 accumulator, y = alpha_w*acc + b,
-//              bf16 round-to-nearest-even, 16-byte stores
+// computation kernel so the output tile is produced once.
+//
+// Persistent kernel, one CTA per SM, 128 x 256 output tiles taken round-robin.
+//   warp 0     producer: per 256-wide K tile, TMA loads of activation codes
+//              [128 x 128 B] and weight codes [256 x 128 B] (128-byte swizzle)
+//              plus 1-D bulk copies of the 512-byte scale atoms; then the
+//              low-rank slab: T (hi/lo bf16) and L2^T/alpha_w (64-byte swizzle)
+//   warp 1     MMA issuer: tcgen05.mma kind::mxf4nvf4 block16 (M128 N256 K64)
+//              per 64-element K block, then kind::f16 (K16) T_hi L2 and T_lo L2
+//              into the same accumulator
+//   warps 2-5  scale writers: read the scale atoms of a K tile from shared
+//              memory and write them into TMEM with tcgen05.st, replicated into
+//              each 32-lane quarter (the layout the block-scaled MMA reads)
+//   warps 6-9  epilogue: tcgen05.ld, y = alpha_w*acc + b, bf16 RNE, 16-byte stores
+// TMEM (512 columns) holds two 256-column accumulators.  Tile j accumulates in
+// acc[j%2] and keeps its scale buffers (2 x 48 columns) in the first 96 columns
+// of acc[(j+1)%2], which the epilogue of tile j-1 releases first; so the
+// epilogue of one tile runs under the main loop of the next.
 #include <algorithm>
 
 #include "ptx.cuh"
@@ -24,15 +30,23 @@ namespace {
 
 using namespace dev;
 
-constexpr int kThreads = 192;
-constexpr int kATile = 128 * 128;  // 128 rows x 128 bytes (256 FP4 along K)
+constexpr int kBN = 256;
+constexpr int kThreads = 320;
+constexpr int kStages = 4;
+constexpr int kATile = 128 * 128;               // 128 rows x 128 bytes (256 FP4 along K)
+constexpr int kBTile = kBN * 128;               // 256 rows x 128 bytes
+constexpr int kSfa = 2048;                      // four 512-byte atoms
+constexpr int kSfb = 2 * 2048;                  // two 128-row blocks x four atoms
+constexpr int kStage = kATile + kBTile + kSfa + kSfb;
+constexpr int kSfCols = 16 + 32;                // TMEM columns of one scale buffer
 
 struct K2Params {
   int M, N, K, r_pad;
   int kt;          // ceil(K / 256)
-  int kb_total;    // K / 64 (scale-atom columns of four 16-groups)
+  int kb_total;    // K / 64
   int nblk_total;  // ceil(N / 128)
   int slab;        // ceil(r_pad / 32)
+  int mtiles, ntiles;
   const uint8_t* xsf;
   const uint8_t* wsf;
   const float* bias;
@@ -42,21 +56,15 @@ struct K2Params {
   uint64_t wait_ns;
 };
 
-template <int BN>
-struct Layout {
-  static constexpr int kB = BN * 128;
-  static constexpr int kSfa = 2048;
-  static constexpr int kSfb = (BN / 128) * 2048;
-  static constexpr int kStage = kATile + kB + kSfa + kSfb;
-  static constexpr int kStages = BN == 256 ? 4 : 6;
-  static constexpr int kSfCols = 16 + 4 * (BN / 32);  // TMEM columns of one scale buffer
-  static constexpr uint32_t kTmemCols = BN + 2 * kSfCols <= 256 ? 256 : 512;
-};
-
 struct K2Shared {
-  uint64_t full[8];
-  uint64_t empty[8];
-  uint64_t acc_full;
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t sf_full[2];
+  uint64_t sf_empty[2];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint64_t sfreg_free[2];
+  uint64_t done;
   uint32_t tmem_base;
   int abort;
 };
@@ -69,32 +77,36 @@ __device__ __noinline__ bool wait_drain(uint64_t* bar, uint32_t parity, uint64_t
   return true;
 }
 
-template <int BN>
 __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
     const __grid_constant__ CUtensorMap map_xq, const __grid_constant__ CUtensorMap map_wq,
     const __grid_constant__ CUtensorMap map_t, const __grid_constant__ CUtensorMap map_l2,
     const K2Params p) {
-  using L = Layout<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  K2Shared* sh = reinterpret_cast<K2Shared*>(smem + L::kStages * L::kStage);
+  K2Shared* sh = reinterpret_cast<K2Shared*>(smem + kStages * kStage);
 
   const uint32_t warp = warp_id(), lane = lane_id();
-  const int m0 = blockIdx.x * 128;
-  const int n0 = blockIdx.y * BN;
-  const int total = p.kt + p.slab;
+  const int ntiles_total = p.mtiles * p.ntiles;
+  const int per_tile = p.kt + p.slab;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < L::kStages; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(&sh->full[s], 1);
-      mbar_init(&sh->empty[s], 1);
+      mbar_init(&sh->empty[s], 1 + 4);  // MMA commit + the four scale writers
     }
-    mbar_init(&sh->acc_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sh->sf_full[b], 4);
+      mbar_init(&sh->sf_empty[b], 1);
+      mbar_init(&sh->acc_full[b], 1);
+      mbar_init(&sh->acc_empty[b], 4);
+      mbar_init(&sh->sfreg_free[b], 4);
+    }
+    mbar_init(&sh->done, 1);
     sh->abort = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(&sh->tmem_base, L::kTmemCols);
+    tmem_alloc(&sh->tmem_base, 512);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -104,6 +116,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
   const uint32_t tmem = sh->tmem_base;
 
   if (warp == 0) {
+    // ------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&map_xq);
       tma_prefetch_desc(&map_wq);
@@ -111,105 +124,195 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
         tma_prefetch_desc(&map_t);
         tma_prefetch_desc(&map_l2);
       }
-      int issued = 0;
-      for (int it = 0; it < total; ++it) {
-        const int s = it % L::kStages;
-        const uint32_t ph = (it / L::kStages) & 1;
-        if (!wait_bounded(&sh->empty[s], ph ^ 1, wc)) break;
-        uint8_t* st = smem + s * L::kStage;
-        if (it < p.kt) {
-          const int nkb = min(4, p.kb_total - 4 * it);
-          int nb_valid = 0;
-          for (int nb = 0; nb < BN / 128; ++nb) nb_valid += (n0 / 128 + nb < p.nblk_total);
-          const uint32_t bytes = kATile + L::kB + 512u * nkb * (1 + nb_valid);
-          mbar_arrive_expect_tx(&sh->full[s], bytes);
-          tma_load_2d(st, &map_xq, &sh->full[s], it * 128, m0);
-          tma_load_2d(st + kATile, &map_wq, &sh->full[s], it * 128, n0);
-          bulk_load(st + kATile + L::kB,
-                    p.xsf + (static_cast<size_t>(m0 / 128) * p.kb_total + 4 * it) * 512, 512u * nkb,
-                    &sh->full[s]);
-          for (int nb = 0; nb < BN / 128; ++nb) {
-            const int nblk = n0 / 128 + nb;
-            if (nblk < p.nblk_total)
-              bulk_load(st + kATile + L::kB + L::kSfa + nb * 2048,
-                        p.wsf + (static_cast<size_t>(nblk) * p.kb_total + 4 * it) * 512, 512u * nkb,
-                        &sh->full[s]);
+      int it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < ntiles_total; t += gridDim.x) {
+        const int m0 = (t % p.mtiles) * 128;
+        const int n0 = (t / p.mtiles) * kBN;
+        int nb_valid = 0;
+        for (int nb = 0; nb < 2; ++nb) nb_valid += (n0 / 128 + nb < p.nblk_total);
+        for (int k = 0; k < per_tile; ++k, ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = (it / kStages) & 1;
+          if (!wait_bounded(&sh->empty[s], ph ^ 1, wc)) {
+            ok = false;
+            break;
           }
-        } else {
-          const int j = it - p.kt;
-          mbar_arrive_expect_tx(&sh->full[s], kATile + BN * 64);
-          tma_load_2d(st, &map_t, &sh->full[s], 64 * j, m0);
-          tma_load_2d(st + kATile, &map_l2, &sh->full[s], 32 * j, n0);
+          uint8_t* st = smem + s * kStage;
+          if (k < p.kt) {
+            const int nkb = min(4, p.kb_total - 4 * k);
+            mbar_arrive_expect_tx(&sh->full[s], kATile + kBTile + 512u * nkb * (1 + nb_valid));
+            tma_load_2d(st, &map_xq, &sh->full[s], k * 128, m0);
+            tma_load_2d(st + kATile, &map_wq, &sh->full[s], k * 128, n0);
+            bulk_load(st + kATile + kBTile,
+                      p.xsf + (static_cast<size_t>(m0 / 128) * p.kb_total + 4 * k) * 512, 512u * nkb,
+                      &sh->full[s]);
+            for (int nb = 0; nb < nb_valid; ++nb)
+              bulk_load(st + kATile + kBTile + kSfa + nb * 2048,
+                        p.wsf + (static_cast<size_t>(n0 / 128 + nb) * p.kb_total + 4 * k) * 512,
+                        512u * nkb, &sh->full[s]);
+          } else {
+            const int j = k - p.kt;
+            mbar_arrive_expect_tx(&sh->full[s], kATile + kBN * 64);
+            tma_load_2d(st, &map_t, &sh->full[s], 64 * j, m0);
+            tma_load_2d(st + kATile, &map_l2, &sh->full[s], 32 * j, n0);
+          }
         }
-        issued = it + 1;
       }
-      if (sh->abort) {
-        for (int i = max(0, issued - L::kStages); i < issued; ++i)
-          wait_drain(&sh->full[i % L::kStages], (i / L::kStages) & 1, p.wait_ns);
+      if (sh->abort) {  // let copies in flight land before the CTA exits
+        for (int i = max(0, it - kStages); i < it; ++i)
+          wait_drain(&sh->full[i % kStages], (i / kStages) & 1, p.wait_ns);
       }
     }
   } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      const uint32_t id_fp4 = idesc_nvfp4(128, BN);
-      const uint32_t id_bf16 = idesc_bf16(128, BN);
-      for (int it = 0; it < total; ++it) {
-        const int s = it % L::kStages;
-        const uint32_t ph = (it / L::kStages) & 1;
-        if (!wait_bounded(&sh->full[s], ph, wc)) break;
+      const uint32_t id_fp4 = idesc_nvfp4(128, kBN);
+      const uint32_t id_bf16 = idesc_bf16(128, kBN);
+      int it = 0, sfi = 0, j = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < ntiles_total; t += gridDim.x, ++j) {
+        const int a = j & 1;
+        if (!wait_bounded(&sh->acc_empty[a], ((j >> 1) & 1) ^ 1, wc)) break;
         tc_fence_after();
-        const uint32_t a_s = smem_u32(smem + s * L::kStage);
-        const uint32_t b_s = a_s + kATile;
-        if (it < p.kt) {
-          const int nkb = min(4, p.kb_total - 4 * it);
-          const uint32_t sfa_t = tmem + BN + (it & 1) * L::kSfCols;
-          const uint32_t sfb_t = sfa_t + 16;
-          const uint32_t sfa_s = b_s + L::kB;
-          const uint32_t sfb_s = sfa_s + L::kSfa;
-          for (int kb = 0; kb < nkb; ++kb) {
-            tmem_cp_sf_atom(sfa_t + 4 * kb, desc_sf_atom(sfa_s + 512 * kb));
-#pragma unroll
-            for (int nb = 0; nb < BN / 128; ++nb)
-              tmem_cp_sf_atom(sfb_t + kb * (BN / 32) + 4 * nb,
-                              desc_sf_atom(sfb_s + nb * 2048 + 512 * kb));
+        const uint32_t acc = tmem + a * 256;
+        const uint32_t sf_region = tmem + (a ^ 1) * 256;
+        for (int k = 0; k < per_tile; ++k, ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = (it / kStages) & 1;
+          if (!wait_bounded(&sh->full[s], ph, wc)) {
+            ok = false;
+            break;
           }
-          for (int kb = 0; kb < nkb; ++kb)
-            mma_nvfp4(tmem, desc_kmajor_sw128(a_s + 32 * kb), desc_kmajor_sw128(b_s + 32 * kb),
-                      id_fp4, sfa_t + 4 * kb, sfb_t + kb * (BN / 32), (it | kb) != 0);
-        } else {
-          const int j = it - p.kt;
+          const uint32_t a_s = smem_u32(smem + s * kStage);
+          const uint32_t b_s = a_s + kATile;
+          if (k < p.kt) {
+            const int b = sfi & 1;
+            if (!wait_bounded(&sh->sf_full[b], (sfi >> 1) & 1, wc)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const int nkb = min(4, p.kb_total - 4 * k);
+            const uint32_t sfa = sf_region + b * kSfCols;
+            const uint32_t sfb = sfa + 16;
+            for (int kb = 0; kb < nkb; ++kb)
+              mma_nvfp4(acc, desc_kmajor_sw128(a_s + 32 * kb), desc_kmajor_sw128(b_s + 32 * kb), id_fp4,
+                        sfa + 4 * kb, sfb + 8 * kb, (k | kb) != 0);
+            mma_commit(&sh->empty[s]);
+            mma_commit(&sh->sf_empty[b]);
+            ++sfi;
+          } else {
+            tc_fence_after();
+            const int jj = k - p.kt;
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            if (32 * j + 16 * c >= p.r_pad) break;
-            const uint64_t bdesc = desc_kmajor_sw64(b_s + 32 * c);
-            mma_bf16(tmem, desc_kmajor_sw128(a_s + 64 * c), bdesc, id_bf16, 1);       // T_hi
-            mma_bf16(tmem, desc_kmajor_sw128(a_s + 64 * c + 32), bdesc, id_bf16, 1);  // T_lo
+            for (int c = 0; c < 2; ++c) {
+              if (32 * jj + 16 * c >= p.r_pad) break;
+              const uint64_t bdesc = desc_kmajor_sw64(b_s + 32 * c);
+              mma_bf16(acc, desc_kmajor_sw128(a_s + 64 * c), bdesc, id_bf16, 1);       // T_hi
+              mma_bf16(acc, desc_kmajor_sw128(a_s + 64 * c + 32), bdesc, id_bf16, 1);  // T_lo
+            }
+            mma_commit(&sh->empty[s]);
           }
         }
-        mma_commit(&sh->empty[s]);
+        if (ok) mma_commit(&sh->acc_full[a]);
       }
-      mma_commit(&sh->acc_full);
+      mma_commit(&sh->done);
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------------ scale writers
+    const int q = warp & 3;
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    int it = 0, sfi = 0, j = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; ok && t < ntiles_total; t += gridDim.x, ++j) {
+      const int a = j & 1;
+      // the scale buffers live in acc[a^1]: wait until the previous tile's
+      // epilogue has read its first 96 columns
+      if (!wait_bounded(&sh->sfreg_free[a ^ 1], ((j - 1) >> 1) & 1, wc)) break;
+      const uint32_t sf_region = tmem + (a ^ 1) * 256 + lane_off;
+      for (int k = 0; k < per_tile; ++k, ++it) {
+        const int s = it % kStages;
+        const uint32_t ph = (it / kStages) & 1;
+        if (k < p.kt) {
+          const int b = sfi & 1;
+          if (!wait_bounded(&sh->sf_empty[b], ((sfi >> 1) & 1) ^ 1, wc) ||
+              !wait_bounded(&sh->full[s], ph, wc)) {
+            ok = false;
+            break;
+          }
+          const uint8_t* sfa_s = smem + s * kStage + kATile + kBTile;
+          const uint8_t* sfb_s = sfa_s + kSfa;
+          uint32_t ra[16], rb[32];
+#pragma unroll
+          for (int kb = 0; kb < 4; ++kb) {
+            const uint4 v = *reinterpret_cast<const uint4*>(sfa_s + kb * 512 + lane * 16);
+            ra[4 * kb] = v.x;
+            ra[4 * kb + 1] = v.y;
+            ra[4 * kb + 2] = v.z;
+            ra[4 * kb + 3] = v.w;
+#pragma unroll
+            for (int nb = 0; nb < 2; ++nb) {
+              const uint4 u = *reinterpret_cast<const uint4*>(sfb_s + nb * 2048 + kb * 512 + lane * 16);
+              rb[8 * kb + 4 * nb] = u.x;
+              rb[8 * kb + 4 * nb + 1] = u.y;
+              rb[8 * kb + 4 * nb + 2] = u.z;
+              rb[8 * kb + 4 * nb + 3] = u.w;
+            }
+          }
+          const uint32_t dst = sf_region + b * kSfCols;
+          tmem_st_x16(dst, ra);
+          tmem_st_x32(dst + 16, rb);
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&sh->sf_full[b]);
+            mbar_arrive(&sh->empty[s]);
+          }
+          ++sfi;
+        } else {
+          if (!wait_bounded(&sh->full[s], ph, wc)) {
+            ok = false;
+            break;
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sh->empty[s]);
+        }
+      }
     }
   } else {
+    // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     const int row = q * 32 + lane;
-    const int m = m0 + row;
-    if (wait_bounded(&sh->acc_full, 0, wc)) {
+    int j = 0;
+    for (int t = blockIdx.x; t < ntiles_total; t += gridDim.x, ++j) {
+      const int a = j & 1;
+      if (!wait_bounded(&sh->acc_full[a], (j >> 1) & 1, wc)) break;
       tc_fence_after();
-      for (int j = 0; j < BN / 32; ++j) {
+      const int m = (t % p.mtiles) * 128 + row;
+      const int n0 = (t / p.mtiles) * kBN;
+      for (int c = 0; c < kBN / 32; ++c) {
         uint32_t r[32];
-        tmem_ld_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + 32 * j, r);
+        tmem_ld_x32(tmem + a * 256 + lane_off + 32 * c, r);
         tmem_ld_wait();
-        const int n = n0 + 32 * j;
+        if (c == 2) {  // columns 0..95 read: the next tile's scale buffers may go there
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sh->sfreg_free[a]);
+        }
+        const int n = n0 + 32 * c;
         if (m < p.M && n < p.N) {
           uint32_t packed[16];
           const float4* b4 = reinterpret_cast<const float4*>(p.bias + n);
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            const float4 b = __ldg(b4 + i);
-            const float y0 = __fadd_rn(__fmul_rn(__uint_as_float(r[4 * i + 0]), p.alpha_w), b.x);
-            const float y1 = __fadd_rn(__fmul_rn(__uint_as_float(r[4 * i + 1]), p.alpha_w), b.y);
-            const float y2 = __fadd_rn(__fmul_rn(__uint_as_float(r[4 * i + 2]), p.alpha_w), b.z);
-            const float y3 = __fadd_rn(__fmul_rn(__uint_as_float(r[4 * i + 3]), p.alpha_w), b.w);
+            const float4 bv = __ldg(b4 + i);
+            const float y0 = __fadd_rn(__fmul_rn(__uint_as_float(r[4 * i + 0]), p.alpha_w), bv.x);
+            const float y1 = __fadd_rn(__fmul_rn(__uint_as_float(r[4 * i + 1]), p.alpha_w), bv.y);
+            const float y2 = __fadd_rn(__fmul_rn(__uint_as_float(r[4 * i + 2]), p.alpha_w), bv.z);
+            const float y3 = __fadd_rn(__fmul_rn(__uint_as_float(r[4 * i + 3]), p.alpha_w), bv.w);
             packed[2 * i] = __bfloat16_as_ushort(__float2bfloat16_rn(y0)) |
                             (uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(y1))) << 16);
             packed[2 * i + 1] = __bfloat16_as_ushort(__float2bfloat16_rn(y2)) |
@@ -222,35 +325,31 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
               dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
         }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->acc_empty[a]);
     }
   }
 
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
-    if (lane == 0) wait_drain(&sh->acc_full, 0, p.wait_ns);
+    if (lane == 0) wait_drain(&sh->done, 0, p.wait_ns);  // every MMA has retired
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, Layout<BN>::kTmemCols);
+    tmem_dealloc(tmem, 512);
   }
 }
 
-template <int BN>
-svdq_status launch_bn(const GemmArgs& a, const CUtensorMap& map_xq, const CUtensorMap& map_wq,
-                      const CUtensorMap& map_t, const CUtensorMap& map_l2, const K2Params& p,
-                      cudaStream_t stream) {
-  using L = Layout<BN>;
-  const size_t smem = 1024 + static_cast<size_t>(L::kStages) * L::kStage + sizeof(K2Shared);
-  static bool attr_set = false;
-  if (!attr_set) {
-    SVDQ_CUDA_TRY(cudaFuncSetAttribute(gemm_w4a4_kernel<BN>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));
-    attr_set = true;
+int num_sms() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
   }
-  dim3 grid((a.M + 127) / 128, (a.N + BN - 1) / BN, 1);
-  gemm_w4a4_kernel<BN><<<grid, kThreads, smem, stream>>>(map_xq, map_wq, map_t, map_l2, p);
-  SVDQ_CUDA_TRY(cudaGetLastError());
-  return SVDQ_OK;
+  return n;
 }
 
 }  // namespace
@@ -265,6 +364,8 @@ svdq_status launch_gemm_w4a4(const GemmArgs& a, cudaStream_t stream) {
   p.kb_total = a.K / 64;
   p.nblk_total = (a.N + 127) / 128;
   p.slab = (a.r_pad + 31) / 32;
+  p.mtiles = (a.M + 127) / 128;
+  p.ntiles = (a.N + kBN - 1) / kBN;
   p.xsf = static_cast<const uint8_t*>(a.xsf);
   p.wsf = a.wsf;
   p.bias = a.bias;
@@ -274,14 +375,9 @@ svdq_status launch_gemm_w4a4(const GemmArgs& a, cudaStream_t stream) {
   p.wait_ns = wait_limit_ns();
   if (!p.err) return fail(SVDQ_ERR_CUDA, "device error word unavailable");
 
-  int bn = a.force_bn;
-  if (bn != 128 && bn != 256) {
-    const long tiles256 = static_cast<long>((a.M + 127) / 128) * ((a.N + 255) / 256);
-    bn = (a.N % 256 == 0 && tiles256 >= 148) ? 256 : 128;
-  }
   CUtensorMap map_xq;
-  svdq_status st = make_tmap_2d(&map_xq, a.xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.K / 2, a.M, a.K / 2,
-                                128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  svdq_status st = make_tmap_2d(&map_xq, a.xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.K / 2, a.M, a.K / 2, 128,
+                                128, CU_TENSOR_MAP_SWIZZLE_128B);
   if (st != SVDQ_OK) return st;
   CUtensorMap map_t = map_xq;
   if (a.r_pad > 0) {
@@ -289,9 +385,20 @@ svdq_status launch_gemm_w4a4(const GemmArgs& a, cudaStream_t stream) {
                       static_cast<uint64_t>(4 * a.r_pad), 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != SVDQ_OK) return st;
   }
-  if (bn == 256)
-    return launch_bn<256>(a, map_xq, *a.map_wq_256, map_t, a.r_pad ? *a.map_l2_256 : map_xq, p, stream);
-  return launch_bn<128>(a, map_xq, *a.map_wq_128, map_t, a.r_pad ? *a.map_l2_128 : map_xq, p, stream);
+  const CUtensorMap& map_l2 = a.r_pad > 0 ? *a.map_l2_256 : map_xq;
+
+  const size_t smem = 1024 + static_cast<size_t>(kStages) * kStage + sizeof(K2Shared);
+  static bool attr_set = false;
+  if (!attr_set) {
+    SVDQ_CUDA_TRY(cudaFuncSetAttribute(gemm_w4a4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem)));
+    attr_set = true;
+  }
+  const int tiles = p.mtiles * p.ntiles;
+  const int grid = std::min(tiles, num_sms());
+  gemm_w4a4_kernel<<<grid, kThreads, smem, stream>>>(map_xq, *a.map_wq_256, map_t, map_l2, p);
+  SVDQ_CUDA_TRY(cudaGetLastError());
+  return SVDQ_OK;
 }
 
 }  // namespace svdq
