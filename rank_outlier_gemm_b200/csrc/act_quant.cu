@@ -6,14 +6,18 @@
 // T = X L1' through distributed shared memory.
 //
 // Per 64-column K tile (one TMA box, 128-byte swizzled rows):
-//   warp 0     TMA producer: X tile [128 x 64] bf16 and L1'^T tile [r_pad x 64]
-//   warp 1     tcgen05.mma kind::f16 (M=128, N=r_pad, K=16 x 4) into TMEM, same
-//              shared-memory X tile as the quantizers read
-//   warps 2-5  thread = row: smoothing multiply, per-16 amax, E4M3 scale,
-//              E2M1 codes; 32 code bytes and one 4-byte scale word per row
+//   warp 0     producer: TMA of the X tile [128 x 64] bf16 and the L1'^T tile
+//              [r_pad x 64], bulk copy of the 64 smoothing multipliers
+//   warp 1     tcgen05.mma kind::f16 (M=128, N=r_pad, K=16 x 4) into TMEM from
+//              the same shared-memory X tile the quantizers read
+//   warps 2-9  quantizers: a thread takes two adjacent 16-groups of one row:
+//              smoothing multiply, amax, E4M3 scale, E2M1 codes; 16 code bytes
+//              and, with its neighbour lane, one 4-byte scale word per row
 // After the K loop the quantizer warps move T from TMEM to shared memory, the
-// cluster syncs, each CTA sums its share of rows over all S partials and writes
-// T as a bf16 hi/lo pair.
+// cluster syncs, each CTA sums its share of rows over all S partials (fixed
+// order) and writes T as a bf16 hi/lo pair.
+#include <cooperative_groups.h>
+
 #include <algorithm>
 
 #include "nvfp4.cuh"
@@ -25,8 +29,10 @@ namespace {
 using namespace dev;
 
 constexpr int kStages = 4;
-constexpr int kThreads = 192;
+constexpr int kQuantWarps = 8;
+constexpr int kThreads = (2 + kQuantWarps) * 32;
 constexpr int kXTile = 128 * 128;  // 128 rows x 64 bf16
+constexpr int kInvTile = 64 * 4;   // 64 fp32 smoothing multipliers
 
 struct K1Params {
   int M, K, r_pad, kt_total, splits;
@@ -60,17 +66,18 @@ __device__ __noinline__ bool wait_drain(uint64_t* bar, uint32_t parity, uint64_t
 }
 
 __device__ __forceinline__ void bar_sync_quant() {
-  asm volatile("bar.sync 1, 128;" ::: "memory");
+  asm volatile("bar.sync 1, %0;" ::"n"(kQuantWarps * 32) : "memory");
 }
 
-__global__ void __launch_bounds__(kThreads) act_quant_lowrank_kernel(
+__global__ void __launch_bounds__(kThreads, 2) act_quant_lowrank_kernel(
     const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_l1,
     const K1Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* xs = smem;
-  uint8_t* l1s = smem + kStages * kXTile;
-  K1Shared* sh = reinterpret_cast<K1Shared*>(l1s + kStages * p.l1_tile);
+  uint8_t* l1s = xs + kStages * kXTile;
+  uint8_t* invs = l1s + kStages * p.l1_tile;
+  K1Shared* sh = reinterpret_cast<K1Shared*>(invs + kStages * kInvTile);
   float* red = reinterpret_cast<float*>(smem);  // reuses the stage buffers after the K loop
   const int red_stride = p.r_pad + 4;
 
@@ -86,7 +93,7 @@ __global__ void __launch_bounds__(kThreads) act_quant_lowrank_kernel(
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sh->full[s], 1);
-      mbar_init(&sh->empty[s], 4 + (lowrank ? 1 : 0));
+      mbar_init(&sh->empty[s], kQuantWarps + (lowrank ? 1 : 0));
     }
     mbar_init(&sh->tfull, 1);
     mbar_init(&sh->never, 1);
@@ -107,7 +114,7 @@ __global__ void __launch_bounds__(kThreads) act_quant_lowrank_kernel(
     if (lane == 0) {
       tma_prefetch_desc(&map_x);
       if (lowrank) tma_prefetch_desc(&map_l1);
-      const uint32_t bytes = kXTile + (lowrank ? p.l1_tile : 0u);
+      const uint32_t bytes = kXTile + (lowrank ? p.l1_tile : 0u) + kInvTile;
       int issued = 0;
       for (int i = 0; i < nt; ++i) {
         const int s = i % kStages;
@@ -117,6 +124,7 @@ __global__ void __launch_bounds__(kThreads) act_quant_lowrank_kernel(
         const int k0 = (t0 + i) * 64;
         tma_load_2d(xs + s * kXTile, &map_x, &sh->full[s], k0, m0);
         if (lowrank) tma_load_2d(l1s + s * p.l1_tile, &map_l1, &sh->full[s], k0, 0);
+        bulk_load(invs + s * kInvTile, p.inv_lam + k0, kInvTile, &sh->full[s]);
         issued = i + 1;
       }
       if (sh->abort) {  // let copies in flight land before the buffers are reused
@@ -143,56 +151,64 @@ __global__ void __launch_bounds__(kThreads) act_quant_lowrank_kernel(
       mma_commit(&sh->tfull);
     }
   } else {
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
-    const int row = q * 32 + lane;
+    // ------------------------------------------------------------ quantizers
+    const int wq = static_cast<int>(warp) - 2;           // 0..7
+    const int row = 16 * wq + static_cast<int>(lane >> 1);
+    const int h = lane & 1;                              // columns [32h, 32h + 32) of the tile
     const int m = m0 + row;
-    if (p.stall) wait_bounded(&sh->never, 0, wc);
+    if (p.stall) wait_warp(&sh->never, 0, wc);
     for (int i = 0; i < nt; ++i) {
       const int s = i % kStages;
       const uint32_t ph = (i / kStages) & 1;
-      if (!wait_bounded(&sh->full[s], ph, wc)) break;
+      if (!wait_warp(&sh->full[s], ph, wc)) break;
       const uint8_t* xrow = xs + s * kXTile + row * 128;
+      const float4* inv4 = reinterpret_cast<const float4*>(invs + s * kInvTile) + 8 * h;
       const int kt = t0 + i;
       const int k0 = kt * 64;
-      uint32_t codes[8];
-      uint32_t sc = 0;
+      float v[32];
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
+      for (int c = 0; c < 4; ++c) {
         // 128-byte swizzle: 16-byte chunk c of row r sits at chunk c ^ (r % 8).
-        const uint4 c0 = *reinterpret_cast<const uint4*>(xrow + (((2 * g) ^ (row & 7)) << 4));
-        const uint4 c1 = *reinterpret_cast<const uint4*>(xrow + (((2 * g + 1) ^ (row & 7)) << 4));
-        const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-        const float4* il = reinterpret_cast<const float4*>(p.inv_lam + k0 + 16 * g);
-        const float4 i0 = __ldg(il), i1 = __ldg(il + 1), i2 = __ldg(il + 2), i3 = __ldg(il + 3);
-        const float inv[16] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w,
-                               i2.x, i2.y, i2.z, i2.w, i3.x, i3.y, i3.z, i3.w};
-        float v[16];
+        const uint4 w = *reinterpret_cast<const uint4*>(xrow + (((4 * h + c) ^ (row & 7)) << 4));
+        const float4 i0 = inv4[2 * c], i1 = inv4[2 * c + 1];
+        const float2 a0 = mul_f32x2(make_float2(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xFFFF0000u)), make_float2(i0.x, i0.y));
+        const float2 a1 = mul_f32x2(make_float2(__uint_as_float(w.y << 16), __uint_as_float(w.y & 0xFFFF0000u)), make_float2(i0.z, i0.w));
+        const float2 a2 = mul_f32x2(make_float2(__uint_as_float(w.z << 16), __uint_as_float(w.z & 0xFFFF0000u)), make_float2(i1.x, i1.y));
+        const float2 a3 = mul_f32x2(make_float2(__uint_as_float(w.w << 16), __uint_as_float(w.w & 0xFFFF0000u)), make_float2(i1.z, i1.w));
+        v[8 * c + 0] = a0.x; v[8 * c + 1] = a0.y; v[8 * c + 2] = a1.x; v[8 * c + 3] = a1.y;
+        v[8 * c + 4] = a2.x; v[8 * c + 5] = a2.y; v[8 * c + 6] = a3.x; v[8 * c + 7] = a3.y;
+      }
+      float g0[16], g1[16];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          v[2 * j] = __fmul_rn(__uint_as_float(w[j] << 16), inv[2 * j]);
-          v[2 * j + 1] = __fmul_rn(__uint_as_float(w[j] & 0xFFFF0000u), inv[2 * j + 1]);
-        }
-        const Fp4Group gq = nvfp4_encode16(v);
-        codes[2 * g] = gq.lo;
-        codes[2 * g + 1] = gq.hi;
-        sc |= gq.scale << (8 * g);
+      for (int j = 0; j < 16; ++j) {
+        g0[j] = v[j];
+        g1[j] = v[16 + j];
       }
-      if (m < p.M) {
-        uint4* dst = reinterpret_cast<uint4*>(p.xq + static_cast<size_t>(m) * (p.K / 2) + k0 / 2);
-        dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
-        dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
-      }
-      const size_t atom = static_cast<size_t>(mb) * p.kt_total + kt;
-      *reinterpret_cast<uint32_t*>(p.xsf + atom * 512 + (row & 31) * 16 + (row >> 5) * 4) = sc;
+      const Fp4Group q0 = nvfp4_encode16(g0);
+      const Fp4Group q1 = nvfp4_encode16(g1);
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sh->empty[s]);
+      if (lane == 0) mbar_arrive(&sh->empty[s]);  // this warp is done reading the stage
+      if (m < p.M) {
+        uint4* dst = reinterpret_cast<uint4*>(p.xq + static_cast<size_t>(m) * (p.K / 2) + k0 / 2 + 16 * h);
+        *dst = make_uint4(q0.lo, q0.hi, q1.lo, q1.hi);
+      }
+      const uint32_t mine = q0.scale | (q1.scale << 8);
+      const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
+      if (h == 0) {
+        const size_t atom = static_cast<size_t>(mb) * p.kt_total + kt;
+        *reinterpret_cast<uint32_t*>(p.xsf + atom * 512 + (row & 31) * 16 + (row >> 5) * 4) =
+            mine | (other << 16);
+      }
     }
     if (lowrank) {
       bar_sync_quant();  // every quantizer is done with the stage buffers
-      if (!sh->abort && wait_bounded(&sh->tfull, 0, wc)) {
+      if (wait_warp(&sh->tfull, 0, wc)) {
         tc_fence_after();
-        float* dst = red + row * red_stride;
-        for (int c = 0; c < p.r_pad; c += 16) {
+        const int q = warp & 3;           // TMEM lane quarter this warp may access
+        const int half = wq >> 2;         // the two warps of a quarter split the 16-column chunks
+        const int trow = q * 32 + static_cast<int>(lane);
+        float* dst = red + trow * red_stride;
+        for (int c = 16 * half; c < p.r_pad; c += 32) {
           uint32_t r[16];
           tmem_ld_x16(tmem + (static_cast<uint32_t>(q * 32) << 16) + c, r);
           tmem_ld_wait();
@@ -207,35 +223,44 @@ __global__ void __launch_bounds__(kThreads) act_quant_lowrank_kernel(
   }
 
   // ---- cluster-wide reduction of the partial T over the K splits
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
   tc_fence_before();
-  cluster_sync_all();
+  cluster.sync();
   if (lowrank && !sh->abort) {
     const int rows_per = (128 + p.splits - 1) / p.splits;
     const int r_lo = split * rows_per;
     const int r_hi = min(128, r_lo + rows_per);
     const int c4n = p.r_pad / 4;
-    const uint32_t red_addr = smem_u32(red);
+    const float* peers[8];
+#pragma unroll
+    for (int qr = 0; qr < 8; ++qr) peers[qr] = cluster.map_shared_rank(red, qr < p.splits ? qr : 0);
     for (int it = threadIdx.x; it < (r_hi - r_lo) * c4n; it += kThreads) {
       const int rr = r_lo + it / c4n;
       const int c = (it % c4n) * 4;
       const int m = m0 + rr;
       if (m >= p.M) continue;
-      const uint32_t off = static_cast<uint32_t>((rr * red_stride + c) * 4);
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int qr = 0; qr < p.splits; ++qr) {
-        const float4 v = ld_dsmem_f4(mapa_shared(red_addr + off, qr));
-        acc.x += v.x;
-        acc.y += v.y;
-        acc.z += v.z;
-        acc.w += v.w;
-      }
+      const int off = rr * red_stride + c;
+      float4 v[8];
+#pragma unroll
+      for (int qr = 0; qr < 8; ++qr)
+        if (qr < p.splits) v[qr] = *reinterpret_cast<const float4*>(peers[qr] + off);
+      float4 acc = v[0];
+#pragma unroll
+      for (int qr = 1; qr < 8; ++qr)
+        if (qr < p.splits) {
+          acc.x += v[qr].x;
+          acc.y += v[qr].y;
+          acc.z += v[qr].z;
+          acc.w += v[qr].w;
+        }
       const float a[4] = {acc.x, acc.y, acc.z, acc.w};
       uint16_t hi[4], lo[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const __nv_bfloat16 h = __float2bfloat16_rn(a[j]);
-        hi[j] = __bfloat16_as_ushort(h);
-        lo[j] = __bfloat16_as_ushort(__float2bfloat16_rn(a[j] - __bfloat162float(h)));
+        const __nv_bfloat16 hb = __float2bfloat16_rn(a[j]);
+        hi[j] = __bfloat16_as_ushort(hb);
+        lo[j] = __bfloat16_as_ushort(__float2bfloat16_rn(a[j] - __bfloat162float(hb)));
       }
       uint16_t* trow = p.T + static_cast<size_t>(m) * (2 * p.r_pad) + 32 * (c / 16) + (c % 16);
       *reinterpret_cast<uint2*>(trow) =
@@ -244,7 +269,7 @@ __global__ void __launch_bounds__(kThreads) act_quant_lowrank_kernel(
           make_uint2(lo[0] | (uint32_t(lo[1]) << 16), lo[2] | (uint32_t(lo[3]) << 16));
     }
   }
-  cluster_sync_all();  // peers are done reading this CTA's partial
+  cluster.sync();  // peers are done reading this CTA's partial
 
   if (warp == 1 && lowrank) {
     if (lane == 0) wait_drain(&sh->tfull, 0, p.wait_ns);  // every MMA has retired
@@ -294,11 +319,11 @@ svdq_status launch_act_quant(const ActArgs& a, cudaStream_t stream) {
   p.tmem_cols = cols;
   if (!p.err) return fail(SVDQ_ERR_CUDA, "device error word unavailable");
 
-  const size_t smem = 1024 + kStages * (kXTile + p.l1_tile) + sizeof(K1Shared);
+  const size_t smem = 1024 + kStages * (kXTile + p.l1_tile + kInvTile) + sizeof(K1Shared);
   static bool attr_set = false;
   if (!attr_set) {
     SVDQ_CUDA_TRY(cudaFuncSetAttribute(act_quant_lowrank_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024));
     attr_set = true;
   }
   cudaLaunchConfig_t cfg = {};

@@ -17,10 +17,11 @@
 //              each 32-lane quarter (the layout the block-scaled MMA reads)
 //   warps 6-9  epilogue: tcgen05.ld, y = alpha_w*acc + b, bf16 RNE, 16-byte stores
 // TMEM (512 columns) holds two 256-column accumulators.  Tile j accumulates in
-// acc[j%2] and keeps its scale buffers (2 x 48 columns) in the first 96 columns
+// acc[j%2] and keeps its scale slots (2 x 48 columns, one K tile each) in the first 96 columns
 // of acc[(j+1)%2], which the epilogue of tile j-1 releases first; so the
 // epilogue of one tile runs under the main loop of the next.
 #include <algorithm>
+#include <cstddef>
 
 #include "ptx.cuh"
 #include "svdq_internal.h"
@@ -38,7 +39,8 @@ constexpr int kBTile = kBN * 128;               // 256 rows x 128 bytes
 constexpr int kSfa = 2048;                      // four 512-byte atoms
 constexpr int kSfb = 2 * 2048;                  // two 128-row blocks x four atoms
 constexpr int kStage = kATile + kBTile + kSfa + kSfb;
-constexpr int kSfCols = 16 + 32;                // TMEM columns of one scale buffer
+constexpr int kSfCols = 16 + 32;                // TMEM columns of one scale slot (one K tile)
+constexpr int kSfSlots = 2;                     // 2 x 48 = 96 columns
 
 struct K2Params {
   int M, N, K, r_pad;
@@ -57,10 +59,11 @@ struct K2Params {
 };
 
 struct K2Shared {
+  alignas(16) float bias[4][kBN];  // one slice per epilogue warp (read as float4)
   uint64_t full[kStages];
   uint64_t empty[kStages];
-  uint64_t sf_full[2];
-  uint64_t sf_empty[2];
+  uint64_t sf_full[kSfSlots];
+  uint64_t sf_empty[kSfSlots];
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
   uint64_t sfreg_free[2];
@@ -77,6 +80,30 @@ __device__ __noinline__ bool wait_drain(uint64_t* bar, uint32_t parity, uint64_t
   return true;
 }
 
+// y = alpha_w * acc + b for 32 consecutive columns of one row, bf16 RNE, 16-byte stores.
+__device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], const float* bias_s, const K2Params& p,
+                                            int m, int n) {
+  if (m >= p.M || n >= p.N) return;
+  uint32_t packed[16];
+  const float4* b4 = reinterpret_cast<const float4*>(bias_s);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 bv = b4[i];
+    const float y0 = __fadd_rn(__fmul_rn(__uint_as_float(r[4 * i + 0]), p.alpha_w), bv.x);
+    const float y1 = __fadd_rn(__fmul_rn(__uint_as_float(r[4 * i + 1]), p.alpha_w), bv.y);
+    const float y2 = __fadd_rn(__fmul_rn(__uint_as_float(r[4 * i + 2]), p.alpha_w), bv.z);
+    const float y3 = __fadd_rn(__fmul_rn(__uint_as_float(r[4 * i + 3]), p.alpha_w), bv.w);
+    packed[2 * i] = __bfloat16_as_ushort(__float2bfloat16_rn(y0)) |
+                    (uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(y1))) << 16);
+    packed[2 * i + 1] = __bfloat16_as_ushort(__float2bfloat16_rn(y2)) |
+                        (uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(y3))) << 16);
+  }
+  uint4* dst = reinterpret_cast<uint4*>(p.Y + static_cast<size_t>(m) * p.N + n);
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    if (n + 8 * i < p.N) dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+}
+
 __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
     const __grid_constant__ CUtensorMap map_xq, const __grid_constant__ CUtensorMap map_wq,
     const __grid_constant__ CUtensorMap map_t, const __grid_constant__ CUtensorMap map_l2,
@@ -84,6 +111,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   K2Shared* sh = reinterpret_cast<K2Shared*>(smem + kStages * kStage);
+  static_assert(offsetof(K2Shared, bias) % 16 == 0, "bias slices are read as float4");
+  static_assert((kStages * kStage) % 1024 == 0, "stage buffers keep 1024-byte alignment");
 
   const uint32_t warp = warp_id(), lane = lane_id();
   const int ntiles_total = p.mtiles * p.ntiles;
@@ -94,9 +123,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
       mbar_init(&sh->full[s], 1);
       mbar_init(&sh->empty[s], 1 + 4);  // MMA commit + the four scale writers
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kSfSlots; ++b) {
       mbar_init(&sh->sf_full[b], 4);
       mbar_init(&sh->sf_empty[b], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
       mbar_init(&sh->acc_full[b], 1);
       mbar_init(&sh->acc_empty[b], 4);
       mbar_init(&sh->sfreg_free[b], 4);
@@ -187,20 +218,20 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
           const uint32_t a_s = smem_u32(smem + s * kStage);
           const uint32_t b_s = a_s + kATile;
           if (k < p.kt) {
-            const int b = sfi & 1;
-            if (!wait_bounded(&sh->sf_full[b], (sfi >> 1) & 1, wc)) {
+            const int nkb = min(4, p.kb_total - 4 * k);
+            const int b = sfi & (kSfSlots - 1);
+            if (!wait_bounded(&sh->sf_full[b], (sfi / kSfSlots) & 1, wc)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            const int nkb = min(4, p.kb_total - 4 * k);
             const uint32_t sfa = sf_region + b * kSfCols;
             const uint32_t sfb = sfa + 16;
             for (int kb = 0; kb < nkb; ++kb)
               mma_nvfp4(acc, desc_kmajor_sw128(a_s + 32 * kb), desc_kmajor_sw128(b_s + 32 * kb), id_fp4,
                         sfa + 4 * kb, sfb + 8 * kb, (k | kb) != 0);
-            mma_commit(&sh->empty[s]);
             mma_commit(&sh->sf_empty[b]);
+            mma_commit(&sh->empty[s]);
             ++sfi;
           } else {
             tc_fence_after();
@@ -229,20 +260,20 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
       const int a = j & 1;
       // the scale buffers live in acc[a^1]: wait until the previous tile's
       // epilogue has read its first 96 columns
-      if (!wait_bounded(&sh->sfreg_free[a ^ 1], ((j - 1) >> 1) & 1, wc)) break;
+      if (!wait_warp(&sh->sfreg_free[a ^ 1], ((j - 1) >> 1) & 1, wc)) break;
       const uint32_t sf_region = tmem + (a ^ 1) * 256 + lane_off;
       for (int k = 0; k < per_tile; ++k, ++it) {
         const int s = it % kStages;
         const uint32_t ph = (it / kStages) & 1;
         if (k < p.kt) {
-          const int b = sfi & 1;
-          if (!wait_bounded(&sh->sf_empty[b], ((sfi >> 1) & 1) ^ 1, wc) ||
-              !wait_bounded(&sh->full[s], ph, wc)) {
+          if (!wait_warp(&sh->full[s], ph, wc)) {
             ok = false;
             break;
           }
           const uint8_t* sfa_s = smem + s * kStage + kATile + kBTile;
           const uint8_t* sfb_s = sfa_s + kSfa;
+          // read the K tile's scale atoms first, then release the stage and
+          // wait for the TMEM slot: only the tcgen05.st is on the MMA's path
           uint32_t ra[16], rb[32];
 #pragma unroll
           for (int kb = 0; kb < 4; ++kb) {
@@ -260,19 +291,23 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
               rb[8 * kb + 4 * nb + 3] = u.w;
             }
           }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sh->empty[s]);
+          const int b = sfi & (kSfSlots - 1);
+          if (!wait_warp(&sh->sf_empty[b], ((sfi / kSfSlots) & 1) ^ 1, wc)) {
+            ok = false;
+            break;
+          }
           const uint32_t dst = sf_region + b * kSfCols;
           tmem_st_x16(dst, ra);
           tmem_st_x32(dst + 16, rb);
           tmem_st_wait();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) {
-            mbar_arrive(&sh->sf_full[b]);
-            mbar_arrive(&sh->empty[s]);
-          }
+          if (lane == 0) mbar_arrive(&sh->sf_full[b]);
           ++sfi;
         } else {
-          if (!wait_bounded(&sh->full[s], ph, wc)) {
+          if (!wait_warp(&sh->full[s], ph, wc)) {
             ok = false;
             break;
           }
@@ -289,41 +324,34 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
     int j = 0;
     for (int t = blockIdx.x; t < ntiles_total; t += gridDim.x, ++j) {
       const int a = j & 1;
-      if (!wait_bounded(&sh->acc_full[a], (j >> 1) & 1, wc)) break;
-      tc_fence_after();
       const int m = (t % p.mtiles) * 128 + row;
       const int n0 = (t / p.mtiles) * kBN;
-      for (int c = 0; c < kBN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld_x32(tmem + a * 256 + lane_off + 32 * c, r);
+      // stage this tile's bias slice (per warp) while the main loop still runs
+      float* bias_s = sh->bias[warp - 6];
+      {
+        const float4* src = reinterpret_cast<const float4*>(p.bias + n0) + 2 * lane;
+        float4* dstb = reinterpret_cast<float4*>(bias_s) + 2 * lane;
+        dstb[0] = __ldg(src);
+        dstb[1] = __ldg(src + 1);
+      }
+      __syncwarp();
+      if (!wait_warp(&sh->acc_full[a], (j >> 1) & 1, wc)) break;
+      tc_fence_after();
+      uint32_t r[3][32];
+#pragma unroll
+      for (int c = 0; c < 3; ++c) tmem_ld_x32(tmem + a * 256 + lane_off + 32 * c, r[c]);
+      tmem_ld_wait();
+      // columns 0..95 read: the next tile's scale slots may go there
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->sfreg_free[a]);
+#pragma unroll
+      for (int c = 0; c < 3; ++c) store_chunk(r[c], bias_s + 32 * c, p, m, n0 + 32 * c);
+      for (int c = 3; c < kBN / 32; ++c) {
+        uint32_t rr[32];
+        tmem_ld_x32(tmem + a * 256 + lane_off + 32 * c, rr);
         tmem_ld_wait();
-        if (c == 2) {  // columns 0..95 read: the next tile's scale buffers may go there
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sh->sfreg_free[a]);
-        }
-        const int n = n0 + 32 * c;
-        if (m < p.M && n < p.N) {
-          uint32_t packed[16];
-          const float4* b4 = reinterpret_cast<const float4*>(p.bias + n);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float4 bv = __ldg(b4 + i);
-            const float y0 = __fadd_rn(__fmul_rn(__uint_as_float(r[4 * i + 0]), p.alpha_w), bv.x);
-            const float y1 = __fadd_rn(__fmul_rn(__uint_as_float(r[4 * i + 1]), p.alpha_w), bv.y);
-            const float y2 = __fadd_rn(__fmul_rn(__uint_as_float(r[4 * i + 2]), p.alpha_w), bv.z);
-            const float y3 = __fadd_rn(__fmul_rn(__uint_as_float(r[4 * i + 3]), p.alpha_w), bv.w);
-            packed[2 * i] = __bfloat16_as_ushort(__float2bfloat16_rn(y0)) |
-                            (uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(y1))) << 16);
-            packed[2 * i + 1] = __bfloat16_as_ushort(__float2bfloat16_rn(y2)) |
-                                (uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(y3))) << 16);
-          }
-          uint4* dst = reinterpret_cast<uint4*>(p.Y + static_cast<size_t>(m) * p.N + n);
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            if (n + 8 * i < p.N)
-              dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
-        }
+        store_chunk(rr, bias_s + 32 * c, p, m, n0 + 32 * c);
       }
       tc_fence_before();
       __syncwarp();

@@ -31,7 +31,11 @@ __device__ __forceinline__ Fp4Group nvfp4_encode16(const float (&v)[16]) {
   const float r = s > 0.0f ? __frcp_rn(s) : 0.0f;
   float t[16];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) t[i] = __fmul_rn(v[i], r);
+  for (int i = 0; i < 16; i += 2) {
+    const float2 m = mul_f32x2(make_float2(v[i], v[i + 1]), make_float2(r, r));
+    t[i] = m.x;
+    t[i + 1] = m.y;
+  }
   g.lo = e2m1_canonical_zero(f32x8_to_e2m1(t[0], t[1], t[2], t[3], t[4], t[5], t[6], t[7]));
   g.hi = e2m1_canonical_zero(f32x8_to_e2m1(t[8], t[9], t[10], t[11], t[12], t[13], t[14], t[15]));
   return g;

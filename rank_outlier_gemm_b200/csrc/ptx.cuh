@@ -76,6 +76,14 @@ static __device__ __noinline__ bool wait_bounded(uint64_t* bar, uint32_t parity,
   }
 }
 
+// wait_bounded for a whole warp: every lane waits, then a vote makes the
+// answer warp-uniform so that warp-collective (.sync.aligned) work after it
+// stays convergent even if the abort flag flips during the wait.
+__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, WaitCtl c) {
+  const bool ok = wait_bounded(bar, parity, c);
+  return __all_sync(0xffffffffu, ok);
+}
+
 // -------------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
@@ -240,7 +248,12 @@ __device__ __forceinline__ void tmem_ld_x32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
 }
-// Each thread of the warp writes 16 / 32 consecutive 32-bit columns of its own lane.
+// Each thread of the warp writes 8 / 16 / 32 consecutive 32-bit columns of its own lane.
+__device__ __forceinline__ void tmem_st_x8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
 __device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
@@ -268,6 +281,14 @@ __device__ __forceinline__ void tmem_ld_wait() {
 }
 
 // ------------------------------------------------------------ conversions
+// Two IEEE round-to-nearest fp32 multiplies in one instruction.
+__device__ __forceinline__ float2 mul_f32x2(float2 a, float2 b) {
+  uint64_t x, y, z;
+  x = (static_cast<uint64_t>(__float_as_uint(a.y)) << 32) | __float_as_uint(a.x);
+  y = (static_cast<uint64_t>(__float_as_uint(b.y)) << 32) | __float_as_uint(b.x);
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(z) : "l"(x), "l"(y));
+  return make_float2(__uint_as_float(static_cast<uint32_t>(z)), __uint_as_float(static_cast<uint32_t>(z >> 32)));
+}
 // E4M3 byte of x: round to nearest even, saturate to 448.
 __device__ __forceinline__ uint32_t f32_to_e4m3_rn_sat(float x) {
   uint16_t r;
