@@ -1,15 +1,22 @@
 """SVDQuant W4A4 + low-rank linear layer for B200 (sm_100a).
 
 The compute lives in ``libsvdq.so`` (CUDA kernels behind the C ABI declared in
-``include/svdq.h``); this package is its ctypes binding.
+``include/svdq.h``); ``binding`` is its ctypes binding.  The binding is loaded
+on first use of any name of this package, so that ``python -m
+rank_outlier_gemm_b200.build`` can (re)build the library without loading it;
+using the package without a built library raises ImportError.
 """
 
-from .binding import *  # noqa: F401,F403
-from .binding import (  # noqa: F401
-    EXPORTED,
-    LIB_PATH,
-    SvdqError,
-    Weights,
-    act_buffers,
-    linear,
-)
+import importlib
+
+
+def __getattr__(name):
+    binding = importlib.import_module(".binding", __name__)
+    try:
+        return getattr(binding, name)
+    except AttributeError:
+        raise AttributeError(f"module {__name__!r} has no attribute {name!r}") from None
+
+
+def __dir__():
+    return sorted(set(globals()) | set(dir(importlib.import_module(".binding", __name__))))
