@@ -170,6 +170,31 @@ svdq_status svdq_forward(const svdq_weights* w, const void* X_bf16, int M, void*
 svdq_status svdq_forward_host(const svdq_weights* w, const void* X_host, int M, void* Y_host,
                               void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * svdq_forward without a workspace, for callers that must not allocate device
+ * memory: code running inside a caching allocator's callbacks, a CUDA graph
+ * capture whose pool forbids new allocations, or a serving loop whose memory
+ * is fully reserved up front.  (The paper has no counterpart; this is a
+ * deployment convenience of this library.)
+ *
+ * The intermediates (activation codes, scales, T) live in one static block of
+ * device memory of at most 32 MiB that every GPU loading the library's device
+ * code keeps until the process exits; layers whose intermediates exceed it
+ * (M*K/2 + ceil(M/128)*128*K/16 + 4*M*r_pad bytes, each rounded up to 256)
+ * are rejected with SVDQ_ERR_INVALID_ARG.  The call allocates nothing: the
+ * first call on a device looks up the block's device address (with that
+ * device current), so make that first call before any stream capture.
+ *
+ * All calls on a device share the one block and leave their intermediates in
+ * it; calls whose kernels overlap on the GPU (other streams, other threads)
+ * race on it and must be serialized by the caller.  Nothing in the block needs
+ * to start at zero.  A device-side wait that runs out is recorded in a static
+ * word that this path does not report; its outputs are then unspecified.
+ *   X_bf16  device, M x K bf16          Y_bf16  device, M x N bf16
+ */
+svdq_status svdq_forward_noalloc(const svdq_weights* w, const void* X_bf16, int M, void* Y_bf16,
+                                 void* stream);
+
 /* Sizes in bytes. */
 size_t svdq_act_codes_bytes(int M, int K);                 /* M * K / 2 */
 size_t svdq_act_sf_bytes(int M, int K);                    /* ceil(M/128)*128 * K/16 */

@@ -45,6 +45,7 @@ _SIGS = {
     "svdq_linear_w4a4": (_i, [_vp, _vp, _vp, _vp, _i, _vp, _vp]),
     "svdq_forward": (_i, [_vp, _vp, _i, _vp, _vp, _sz, _vp]),
     "svdq_forward_host": (_i, [_vp, _vp, _i, _vp, _vp, _sz, _vp]),
+    "svdq_forward_noalloc": (_i, [_vp, _vp, _i, _vp, _vp]),
     "svdq_act_codes_bytes": (_sz, [_i, _i]),
     "svdq_act_sf_bytes": (_sz, [_i, _i]),
     "svdq_lowrank_bytes": (_sz, [_vp, _i]),
@@ -207,6 +208,12 @@ def svdq_forward_host(w: Weights, X_host: torch.Tensor, Y_host: torch.Tensor, wo
     _check(_lib.svdq_forward_host(w.handle, X_host.data_ptr(), X_host.shape[0], Y_host.data_ptr(),
                                   _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
                                   _stream(stream)), "svdq_forward_host")
+
+
+def svdq_forward_noalloc(w: Weights, X: torch.Tensor, Y: torch.Tensor, stream=None) -> None:
+    """svdq_forward with the intermediates in the library's static device block (no allocation)."""
+    _check(_lib.svdq_forward_noalloc(w.handle, _dev(X, "X"), X.shape[0], _dev(Y, "Y"), _stream(stream)),
+           "svdq_forward_noalloc")
 
 
 def svdq_act_codes_bytes(M: int, K: int) -> int:

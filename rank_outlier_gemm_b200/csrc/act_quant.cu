@@ -310,7 +310,7 @@ svdq_status launch_act_quant(const ActArgs& a, cudaStream_t stream) {
   p.xq = a.xq;
   p.xsf = a.xsf;
   p.T = a.T;
-  p.err = device_error_word();
+  p.err = a.err ? a.err : device_error_word();
   p.wait_ns = wait_limit_ns();
   p.stall = a.stall;
   p.l1_tile = static_cast<uint32_t>(a.r_pad) * 128u;

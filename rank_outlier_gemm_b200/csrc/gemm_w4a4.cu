@@ -399,7 +399,7 @@ svdq_status launch_gemm_w4a4(const GemmArgs& a, cudaStream_t stream) {
   p.bias = a.bias;
   p.alpha_w = a.alpha_w;
   p.Y = static_cast<uint16_t*>(a.Y);
-  p.err = device_error_word();
+  p.err = a.err ? a.err : device_error_word();
   p.wait_ns = wait_limit_ns();
   if (!p.err) return fail(SVDQ_ERR_CUDA, "device error word unavailable");
 

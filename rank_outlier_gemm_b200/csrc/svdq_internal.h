@@ -48,6 +48,7 @@ struct ActArgs {
   uint16_t* T;              // device [M, 2 r_pad] bf16 (hi/lo chunks)
   int stall;                // test hook: a wait that never completes
   int splits;               // K-splits per 128-row block (0 = automatic)
+  int* err = nullptr;       // device error word (nullptr = the device's default word)
 };
 svdq_status launch_act_quant(const ActArgs& a, cudaStream_t stream);
 
@@ -65,6 +66,7 @@ struct GemmArgs {
   float alpha_w;
   void* Y;                  // device bf16 [M, N]
   int force_bn;             // 0 = automatic, else 128 or 256
+  int* err = nullptr;       // device error word (nullptr = the device's default word)
 };
 svdq_status launch_gemm_w4a4(const GemmArgs& a, cudaStream_t stream);
 
