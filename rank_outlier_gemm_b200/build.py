@@ -40,8 +40,6 @@ def _compile(nvcc: str, src: str, verbose: bool) -> str:
     cmd = [nvcc, *ARCH, *COMMON, "-c", src, "-o", obj]
     if src.endswith(".cu") and verbose:
         cmd += ["-Xptxas", "-v"]
-    if src.endswith(".cpp"):
-        cmd += ["-x", "cu"] if False else []
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"nvcc failed for {src}:\n{r.stdout}\n{r.stderr}")

@@ -19,6 +19,9 @@
 #include <cooperative_groups.h>
 
 #include <algorithm>
+#include <map>
+#include <mutex>
+#include <utility>
 
 #include "nvfp4.cuh"
 #include "svdq_internal.h"
@@ -279,12 +282,56 @@ __global__ void __launch_bounds__(kThreads, 2) act_quant_lowrank_kernel(
   }
 }
 
-int auto_splits(int mblocks, int kt_total) {
-  // Aim for about two CTAs per SM (148 SMs) while keeping >= 4 K tiles per CTA.
-  int s = (2 * 148 + mblocks - 1) / mblocks;
-  s = std::min(s, 8);
-  s = std::min(s, std::max(1, kt_total / 4));
-  return std::max(1, std::min(s, kt_total));
+// Clusters of this kernel that fit on the device at once for a K-split of S
+// (cluster = S CTAs); cached per (S, shared memory size).
+int max_active_clusters(int S, size_t smem) {
+  static std::mutex mu;
+  static std::map<std::pair<int, size_t>, int> cache;
+  std::lock_guard<std::mutex> lk(mu);
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const auto key = std::make_pair(S + 16 * dev, smem);
+  auto it = cache.find(key);
+  if (it != cache.end()) return it->second;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1, S, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = S;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, act_quant_lowrank_kernel, &cfg) != cudaSuccess || n < 1) {
+    cudaGetLastError();
+    n = 1;
+  }
+  cache[key] = n;
+  return n;
+}
+
+// K-split for `mblocks` row blocks of `kt_total` 64-column tiles.  The T
+// reduction needs the S CTAs of a row block in one cluster, and clusters are
+// placed one CTA per SM within a GPC, so splitting more only pays while the
+// clusters still fit: the cost is (waves of clusters) x (tiles per CTA), ties
+// going to the larger split (more CTAs in flight).  At least 4 tiles per CTA.
+int auto_splits(int mblocks, int kt_total, size_t smem) {
+  const int s_max = std::max(1, std::min(8, kt_total / 4));
+  int best = 1;
+  long best_cost = -1;
+  for (int S = 1; S <= s_max; ++S) {
+    const int fit = max_active_clusters(S, smem);
+    const long waves = (mblocks + fit - 1) / fit;
+    const long cost = waves * ((kt_total + S - 1) / S);
+    if (best_cost < 0 || cost <= best_cost) {
+      best_cost = cost;
+      best = S;
+    }
+  }
+  return best;
 }
 
 }  // namespace
@@ -292,7 +339,17 @@ int auto_splits(int mblocks, int kt_total) {
 svdq_status launch_act_quant(const ActArgs& a, cudaStream_t stream) {
   const int mblocks = (a.M + 127) / 128;
   const int kt_total = a.K / 64;
-  int splits = a.splits > 0 ? std::min(std::min(a.splits, 8), kt_total) : auto_splits(mblocks, kt_total);
+  const uint32_t l1_tile = static_cast<uint32_t>(a.r_pad) * 128u;
+  const size_t smem = 1024 + kStages * (kXTile + l1_tile + kInvTile) + sizeof(K1Shared);
+  static bool attr_set[64] = {};  // per device: the attribute is set on the current one
+  int cur_dev = 0;
+  SVDQ_CUDA_TRY(cudaGetDevice(&cur_dev));
+  if (cur_dev < 0 || cur_dev >= 64 || !attr_set[cur_dev]) {
+    SVDQ_CUDA_TRY(cudaFuncSetAttribute(act_quant_lowrank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024));
+    if (cur_dev >= 0 && cur_dev < 64) attr_set[cur_dev] = true;
+  }
+  const int splits = a.splits > 0 ? std::min(std::min(a.splits, 8), kt_total)
+                                   : auto_splits(mblocks, kt_total, smem);
 
   CUtensorMap map_x;
   svdq_status st = make_tmap_2d(&map_x, a.X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.K, a.M,
@@ -313,19 +370,12 @@ svdq_status launch_act_quant(const ActArgs& a, cudaStream_t stream) {
   p.err = a.err ? a.err : device_error_word();
   p.wait_ns = wait_limit_ns();
   p.stall = a.stall;
-  p.l1_tile = static_cast<uint32_t>(a.r_pad) * 128u;
+  p.l1_tile = l1_tile;
   uint32_t cols = 32;
   while (cols < static_cast<uint32_t>(a.r_pad)) cols <<= 1;
   p.tmem_cols = cols;
   if (!p.err) return fail(SVDQ_ERR_CUDA, "device error word unavailable");
 
-  const size_t smem = 1024 + kStages * (kXTile + p.l1_tile + kInvTile) + sizeof(K1Shared);
-  static bool attr_set = false;
-  if (!attr_set) {
-    SVDQ_CUDA_TRY(cudaFuncSetAttribute(act_quant_lowrank_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024));
-    attr_set = true;
-  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(mblocks, splits, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);

@@ -5,13 +5,15 @@
 // computation kernel so the output tile is produced once.
 //
 // Persistent kernel, one CTA per SM, 128 x 256 output tiles taken round-robin.
-//   warp 0     producer: per 256-wide K tile, TMA loads of activation codes
-//              [128 x 128 B] and weight codes [256 x 128 B] (128-byte swizzle)
-//              plus 1-D bulk copies of the 512-byte scale atoms; then the
-//              low-rank slab: T (hi/lo bf16) and L2^T/alpha_w (64-byte swizzle)
-//   warp 1     MMA issuer: tcgen05.mma kind::mxf4nvf4 block16 (M128 N256 K64)
-//              per 64-element K block, then kind::f16 (K16) T_hi L2 and T_lo L2
-//              into the same accumulator
+//   warp 0     producer: per tile, first the low-rank slab -- T (hi/lo bf16)
+//              and L2^T/alpha_w (64-byte swizzle) -- then per 256-wide K tile,
+//              TMA loads of activation codes [128 x 128 B] and weight codes
+//              [256 x 128 B] (128-byte swizzle) plus 1-D bulk copies of the
+//              512-byte scale atoms
+//   warp 1     MMA issuer: kind::f16 (K16) T_hi L2 and T_lo L2, then
+//              tcgen05.mma kind::mxf4nvf4 block16 (M128 N256 K64) per 64-element
+//              K block, all into the same accumulator.  For a K tile it waits
+//              only for the scale writers, which have seen its data land
 //   warps 2-5  scale writers: read the scale atoms of a K tile from shared
 //              memory and write them into TMEM with tcgen05.st, replicated into
 //              each 32-lane quarter (the layout the block-scaled MMA reads)
@@ -19,7 +21,8 @@
 // TMEM (512 columns) holds two 256-column accumulators.  Tile j accumulates in
 // acc[j%2] and keeps its scale slots (2 x 48 columns, one K tile each) in the first 96 columns
 // of acc[(j+1)%2], which the epilogue of tile j-1 releases first; so the
-// epilogue of one tile runs under the main loop of the next.
+// epilogue of one tile runs under the main loop of the next, and the slab MMAs,
+// which need no scales, keep the tensor pipe busy during that hand-over.
 #include <algorithm>
 #include <cstddef>
 
@@ -54,6 +57,7 @@ struct K2Params {
   const float* bias;
   float alpha_w;
   uint16_t* Y;
+  int y32;         // Y is 32-byte aligned: one 32-byte store per 16 columns
   int* err;
   uint64_t wait_ns;
 };
@@ -80,7 +84,8 @@ __device__ __noinline__ bool wait_drain(uint64_t* bar, uint32_t parity, uint64_t
   return true;
 }
 
-// y = alpha_w * acc + b for 32 consecutive columns of one row, bf16 RNE, 16-byte stores.
+// y = alpha_w * acc + b for 32 consecutive columns of one row, bf16 RNE.  Each
+// lane writes whole 32-byte sectors when Y allows it (else 16-byte halves).
 __device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], const float* bias_s, const K2Params& p,
                                             int m, int n) {
   if (m >= p.M || n >= p.N) return;
@@ -98,10 +103,18 @@ __device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], const float
     packed[2 * i + 1] = __bfloat16_as_ushort(__float2bfloat16_rn(y2)) |
                         (uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(y3))) << 16);
   }
-  uint4* dst = reinterpret_cast<uint4*>(p.Y + static_cast<size_t>(m) * p.N + n);
+  uint16_t* dst = p.Y + static_cast<size_t>(m) * p.N + n;
+  if (p.y32) {
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
-    if (n + 8 * i < p.N) dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+    for (int i = 0; i < 2; ++i)
+      if (n + 16 * i < p.N) st_global_v8(dst + 16 * i, &packed[8 * i]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (n + 8 * i < p.N)
+        *reinterpret_cast<uint4*>(dst + 8 * i) =
+            make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+  }
 }
 
 __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
@@ -170,20 +183,21 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
             break;
           }
           uint8_t* st = smem + s * kStage;
-          if (k < p.kt) {
-            const int nkb = min(4, p.kb_total - 4 * k);
+          if (k >= p.slab) {
+            const int kk = k - p.slab;
+            const int nkb = min(4, p.kb_total - 4 * kk);
             mbar_arrive_expect_tx(&sh->full[s], kATile + kBTile + 512u * nkb * (1 + nb_valid));
-            tma_load_2d(st, &map_xq, &sh->full[s], k * 128, m0);
-            tma_load_2d(st + kATile, &map_wq, &sh->full[s], k * 128, n0);
+            tma_load_2d(st, &map_xq, &sh->full[s], kk * 128, m0);
+            tma_load_2d(st + kATile, &map_wq, &sh->full[s], kk * 128, n0);
             bulk_load(st + kATile + kBTile,
-                      p.xsf + (static_cast<size_t>(m0 / 128) * p.kb_total + 4 * k) * 512, 512u * nkb,
+                      p.xsf + (static_cast<size_t>(m0 / 128) * p.kb_total + 4 * kk) * 512, 512u * nkb,
                       &sh->full[s]);
             for (int nb = 0; nb < nb_valid; ++nb)
               bulk_load(st + kATile + kBTile + kSfa + nb * 2048,
-                        p.wsf + (static_cast<size_t>(n0 / 128 + nb) * p.kb_total + 4 * k) * 512,
+                        p.wsf + (static_cast<size_t>(n0 / 128 + nb) * p.kb_total + 4 * kk) * 512,
                         512u * nkb, &sh->full[s]);
           } else {
-            const int j = k - p.kt;
+            const int j = k;
             mbar_arrive_expect_tx(&sh->full[s], kATile + kBN * 64);
             tma_load_2d(st, &map_t, &sh->full[s], 64 * j, m0);
             tma_load_2d(st + kATile, &map_l2, &sh->full[s], 32 * j, n0);
@@ -200,6 +214,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
     if (lane == 0) {
       const uint32_t id_fp4 = idesc_nvfp4(128, kBN);
       const uint32_t id_bf16 = idesc_bf16(128, kBN);
+      // descriptors of stage 0; stage s starts kStage bytes further (the start
+      // address field counts 16-byte units)
+      const uint32_t stage0 = smem_u32(smem);
+      const uint64_t da0 = desc_kmajor_sw128(stage0);
+      const uint64_t db0 = desc_kmajor_sw128(stage0 + kATile);
+      const uint64_t dl0 = desc_kmajor_sw64(stage0 + kATile);
       int it = 0, sfi = 0, j = 0;
       bool ok = true;
       for (int t = blockIdx.x; ok && t < ntiles_total; t += gridDim.x, ++j) {
@@ -208,18 +228,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
         tc_fence_after();
         const uint32_t acc = tmem + a * 256;
         const uint32_t sf_region = tmem + (a ^ 1) * 256;
+        uint32_t accum = 0;  // the tile's first MMA overwrites the accumulator
         for (int k = 0; k < per_tile; ++k, ++it) {
           const int s = it % kStages;
           const uint32_t ph = (it / kStages) & 1;
-          if (!wait_bounded(&sh->full[s], ph, wc)) {
-            ok = false;
-            break;
-          }
-          const uint32_t a_s = smem_u32(smem + s * kStage);
-          const uint32_t b_s = a_s + kATile;
-          if (k < p.kt) {
-            const int nkb = min(4, p.kb_total - 4 * k);
+          const uint64_t soff = static_cast<uint64_t>(s * (kStage >> 4));
+          if (k >= p.slab) {
+            const int nkb = min(4, p.kb_total - 4 * (k - p.slab));
             const int b = sfi & (kSfSlots - 1);
+            // the writers waited for this stage's data before publishing its scales
             if (!wait_bounded(&sh->sf_full[b], (sfi / kSfSlots) & 1, wc)) {
               ok = false;
               break;
@@ -227,21 +244,29 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
             tc_fence_after();
             const uint32_t sfa = sf_region + b * kSfCols;
             const uint32_t sfb = sfa + 16;
-            for (int kb = 0; kb < nkb; ++kb)
-              mma_nvfp4(acc, desc_kmajor_sw128(a_s + 32 * kb), desc_kmajor_sw128(b_s + 32 * kb), id_fp4,
-                        sfa + 4 * kb, sfb + 8 * kb, (k | kb) != 0);
+#pragma unroll
+            for (int kb = 0; kb < 4; ++kb) {
+              if (kb < nkb) {
+                mma_nvfp4(acc, da0 + soff + 2 * kb, db0 + soff + 2 * kb, id_fp4, sfa + 4 * kb, sfb + 8 * kb, accum);
+                accum = 1;
+              }
+            }
             mma_commit(&sh->sf_empty[b]);
             mma_commit(&sh->empty[s]);
             ++sfi;
           } else {
+            if (!wait_bounded(&sh->full[s], ph, wc)) {
+              ok = false;
+              break;
+            }
             tc_fence_after();
-            const int jj = k - p.kt;
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
-              if (32 * jj + 16 * c >= p.r_pad) break;
-              const uint64_t bdesc = desc_kmajor_sw64(b_s + 32 * c);
-              mma_bf16(acc, desc_kmajor_sw128(a_s + 64 * c), bdesc, id_bf16, 1);       // T_hi
-              mma_bf16(acc, desc_kmajor_sw128(a_s + 64 * c + 32), bdesc, id_bf16, 1);  // T_lo
+              if (32 * k + 16 * c >= p.r_pad) break;
+              const uint64_t ldesc = dl0 + soff + 2 * c;
+              mma_bf16(acc, da0 + soff + 4 * c, ldesc, id_bf16, accum);      // T_hi
+              mma_bf16(acc, da0 + soff + 4 * c + 2, ldesc, id_bf16, 1);      // T_lo
+              accum = 1;
             }
             mma_commit(&sh->empty[s]);
           }
@@ -258,14 +283,19 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
     bool ok = true;
     for (int t = blockIdx.x; ok && t < ntiles_total; t += gridDim.x, ++j) {
       const int a = j & 1;
-      // the scale buffers live in acc[a^1]: wait until the previous tile's
-      // epilogue has read its first 96 columns
-      if (!wait_warp(&sh->sfreg_free[a ^ 1], ((j - 1) >> 1) & 1, wc)) break;
       const uint32_t sf_region = tmem + (a ^ 1) * 256 + lane_off;
       for (int k = 0; k < per_tile; ++k, ++it) {
         const int s = it % kStages;
         const uint32_t ph = (it / kStages) & 1;
-        if (k < p.kt) {
+        if (k == p.slab) {
+          // the scale buffers live in acc[a^1]: wait until the previous tile's
+          // epilogue has read its first 96 columns
+          if (!wait_warp(&sh->sfreg_free[a ^ 1], ((j - 1) >> 1) & 1, wc)) {
+            ok = false;
+            break;
+          }
+        }
+        if (k >= p.slab) {
           if (!wait_warp(&sh->full[s], ph, wc)) {
             ok = false;
             break;
@@ -399,6 +429,8 @@ svdq_status launch_gemm_w4a4(const GemmArgs& a, cudaStream_t stream) {
   p.bias = a.bias;
   p.alpha_w = a.alpha_w;
   p.Y = static_cast<uint16_t*>(a.Y);
+  // N % 16 == 0, so every 16-column piece starts 32 bytes after the last
+  p.y32 = (reinterpret_cast<uintptr_t>(a.Y) & 31u) == 0;
   p.err = a.err ? a.err : device_error_word();
   p.wait_ns = wait_limit_ns();
   if (!p.err) return fail(SVDQ_ERR_CUDA, "device error word unavailable");
@@ -416,11 +448,12 @@ svdq_status launch_gemm_w4a4(const GemmArgs& a, cudaStream_t stream) {
   const CUtensorMap& map_l2 = a.r_pad > 0 ? *a.map_l2_256 : map_xq;
 
   const size_t smem = 1024 + static_cast<size_t>(kStages) * kStage + sizeof(K2Shared);
-  static bool attr_set = false;
-  if (!attr_set) {
-    SVDQ_CUDA_TRY(cudaFuncSetAttribute(gemm_w4a4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem)));
-    attr_set = true;
+  static bool attr_set[64] = {};  // per device: the attribute is set on the current one
+  int cur_dev = 0;
+  SVDQ_CUDA_TRY(cudaGetDevice(&cur_dev));
+  if (cur_dev < 0 || cur_dev >= 64 || !attr_set[cur_dev]) {
+    SVDQ_CUDA_TRY(cudaFuncSetAttribute(gemm_w4a4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));
+    if (cur_dev >= 0 && cur_dev < 64) attr_set[cur_dev] = true;
   }
   const int tiles = p.mtiles * p.ntiles;
   const int grid = std::min(tiles, num_sms());

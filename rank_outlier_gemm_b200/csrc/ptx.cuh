@@ -27,6 +27,13 @@ __device__ __forceinline__ uint64_t globaltimer() {
   return t;
 }
 
+// One 32-byte global store of eight 32-bit words (address 32-byte aligned).
+__device__ __forceinline__ void st_global_v8(void* dst, const uint32_t* w) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(w[0]), "r"(w[1]),
+               "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
@@ -60,10 +67,10 @@ struct WaitCtl {
   volatile int* abort; // CTA-wide abort flag (shared)
 };
 
-// Waits for the phase of `bar` with parity `parity` to complete.  Returns false
-// if the CTA is aborting or the wait ran past its limit (then it aborts).
-static __device__ __noinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, WaitCtl c) {
-  if (mbar_try_wait(bar, parity)) return true;
+// Slow path of wait_bounded: polls until the phase completes, the CTA aborts or
+// the time limit passes (then it aborts).  Out of line so that the common case,
+// a phase that is already complete, costs one try_wait and no call.
+static __device__ __noinline__ bool wait_bounded_slow(uint64_t* bar, uint32_t parity, WaitCtl c) {
   const uint64_t t0 = globaltimer();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -76,10 +83,17 @@ static __device__ __noinline__ bool wait_bounded(uint64_t* bar, uint32_t parity,
   }
 }
 
+// Waits for the phase of `bar` with parity `parity` to complete.  Returns false
+// if the CTA is aborting or the wait ran past its limit (then it aborts).
+__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, const WaitCtl& c) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return wait_bounded_slow(bar, parity, c);
+}
+
 // wait_bounded for a whole warp: every lane waits, then a vote makes the
 // answer warp-uniform so that warp-collective (.sync.aligned) work after it
 // stays convergent even if the abort flag flips during the wait.
-__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, WaitCtl c) {
+__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, const WaitCtl& c) {
   const bool ok = wait_bounded(bar, parity, c);
   return __all_sync(0xffffffffu, ok);
 }

@@ -148,6 +148,23 @@ def test_forward_entry_points_agree():
     np.testing.assert_array_equal(Yh.float().numpy(), Y2)
 
 
+def test_output_only_16_byte_aligned():
+    """Y that is 16- but not 32-byte aligned takes the 16-byte store path; the
+    values are the same as with an aligned Y (and rows/columns stay in place)."""
+    L = G.lib()
+    t, prep = _case_prep("pixart/mlp_up", 300)
+    w = G.weights_from_oracle(prep)
+    Y_ref, (xq, xsf, T) = G.run_layer(w, t.X_bits)
+    M, N = t.X_bits.shape[0], w.info["N"]
+    buf = torch.full((M * N + 16,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    assert buf.data_ptr() % 32 == 0
+    Y = buf[8:8 + M * N].view(M, N)  # 16 bytes past a 32-byte boundary
+    L.svdq_linear_w4a4(w, xq, xsf, T, M, Y)
+    assert L.svdq_check_device_errors() == 0
+    np.testing.assert_array_equal(Y.float().cpu().numpy(), Y_ref)
+    assert torch.isnan(buf[:8].float()).all() and torch.isnan(buf[8 + M * N:].float()).all()
+
+
 def test_library_prepare_invariants():
     """The library's own host SVD split: inv_lam as the oracle's, L1 L2 + R
     reconstructs W_hat, and the split is near the Eckart-Young optimum."""
