@@ -247,6 +247,18 @@ svdq_status svdq_check_device_errors(void* stream);
 svdq_status svdq_debug_launch_stalled_act(const svdq_weights* w, const void* X_bf16, int M,
                                           void* xq, void* xsf, void* T, void* stream);
 
+/*
+ * Device self-test of the NVFP4 group encoder's exact shortcuts (both kernels
+ * use them; SVDQuant App. D fixes the codec as IEEE fp32 division by qmax = 6
+ * and reciprocal of the decoded E4M3 scale).  Compares, on the current device,
+ * the fused division by 6 with IEEE division for every fp32 mantissa at
+ * exponents -100..12, and the table reciprocal with the IEEE reciprocal for
+ * every positive finite E4M3 byte.  Synchronous; writes the number of
+ * mismatches (0 when the shortcuts are exact) to *mismatches.
+ * SVDQ_ERR_INVALID_ARG for a null pointer, SVDQ_ERR_UNSUPPORTED_DEVICE off sm_100.
+ */
+svdq_status svdq_selftest_codec(unsigned int* mismatches);
+
 /* Message for the last failed call on this thread ("" if none). */
 const char* svdq_last_error(void);
 

@@ -57,6 +57,7 @@ _SIGS = {
     "svdq_weights_destroy": (_i, [_vp]),
     "svdq_set_wait_limit_ns": (None, [ctypes.c_uint64]),
     "svdq_check_device_errors": (_i, [_vp]),
+    "svdq_selftest_codec": (_i, [ctypes.POINTER(ctypes.c_uint)]),
     "svdq_debug_launch_stalled_act": (_i, [_vp, _vp, _i, _vp, _vp, _vp, _vp]),
     "svdq_last_error": (ctypes.c_char_p, []),
     "svdq_version": (ctypes.c_char_p, []),
@@ -258,6 +259,13 @@ def svdq_weights_export(w: Weights, residual: bool = False) -> dict:
 
 def svdq_set_wait_limit_ns(ns: int) -> None:
     _lib.svdq_set_wait_limit_ns(int(ns))
+
+
+def svdq_selftest_codec() -> int:
+    """Mismatch count of the encoder's exact division/reciprocal shortcuts on the current device."""
+    out = ctypes.c_uint(0)
+    _check(_lib.svdq_selftest_codec(ctypes.byref(out)), "svdq_selftest_codec")
+    return int(out.value)
 
 
 def svdq_check_device_errors(stream=None) -> int:

@@ -51,6 +51,7 @@ struct K1Params {
 };
 
 struct K1Shared {
+  float rcp_tbl[16];  // reciprocals of the E4M3 mantissa patterns (see nvfp4.cuh)
   uint64_t full[kStages];
   uint64_t empty[kStages];
   uint64_t tfull;
@@ -103,6 +104,7 @@ __global__ void __launch_bounds__(kThreads, 2) act_quant_lowrank_kernel(
     sh->abort = 0;
     fence_barrier_init();
   }
+  if (threadIdx.x < 16) sh->rcp_tbl[threadIdx.x] = rcp_table_entry(static_cast<int>(threadIdx.x));
   if (warp == 1 && lowrank) {
     tmem_alloc(&sh->tmem_base, p.tmem_cols);
     tmem_relinquish();
@@ -187,8 +189,8 @@ __global__ void __launch_bounds__(kThreads, 2) act_quant_lowrank_kernel(
         g0[j] = v[j];
         g1[j] = v[16 + j];
       }
-      const Fp4Group q0 = nvfp4_encode16(g0);
-      const Fp4Group q1 = nvfp4_encode16(g1);
+      const Fp4Group q0 = nvfp4_encode16(g0, sh->rcp_tbl);
+      const Fp4Group q1 = nvfp4_encode16(g1, sh->rcp_tbl);
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh->empty[s]);  // this warp is done reading the stage
       if (m < p.M) {

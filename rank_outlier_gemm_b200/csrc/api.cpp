@@ -357,6 +357,12 @@ svdq_status svdq_debug_launch_stalled_act(const svdq_weights* w, const void* X_b
   return launch_act_quant(a, static_cast<cudaStream_t>(stream));
 }
 
+svdq_status svdq_selftest_codec(unsigned int* mismatches) {
+  if (!mismatches) return fail(SVDQ_ERR_INVALID_ARG, "mismatches is null");
+  SVDQ_TRY(check_device());
+  return selftest_codec(mismatches);
+}
+
 svdq_status svdq_linear_w4a4(const svdq_weights* w, const void* xq, const void* xsf, const void* T, int M,
                              void* Y_bf16, void* stream) {
   SVDQ_TRY(check_runtime(w, M));

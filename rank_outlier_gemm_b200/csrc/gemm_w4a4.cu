@@ -244,13 +244,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
             tc_fence_after();
             const uint32_t sfa = sf_region + b * kSfCols;
             const uint32_t sfb = sfa + 16;
-#pragma unroll
-            for (int kb = 0; kb < 4; ++kb) {
-              if (kb < nkb) {
-                mma_nvfp4(acc, da0 + soff + 2 * kb, db0 + soff + 2 * kb, id_fp4, sfa + 4 * kb, sfb + 8 * kb, accum);
-                accum = 1;
-              }
+            const uint64_t adesc = da0 + soff, bdesc = db0 + soff;
+            if (nkb == 4) {
+              mma_nvfp4_x4(acc, adesc, bdesc, id_fp4, sfa, sfb, accum);
+            } else {  // K tail: fewer than four 64-element blocks
+              for (int kb = 0; kb < nkb; ++kb)
+                mma_nvfp4(acc, adesc + 2 * kb, bdesc + 2 * kb, id_fp4, sfa + 4 * kb, sfb + 8 * kb, kb ? 1u : accum);
             }
+            accum = 1;
             mma_commit(&sh->sf_empty[b]);
             mma_commit(&sh->empty[s]);
             ++sfi;

@@ -225,6 +225,26 @@ __device__ __forceinline__ void mma_nvfp4(uint32_t d_tmem, uint64_t a, uint64_t 
       "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
       : "memory");
 }
+// Four block-scaled MMAs over one 256-wide K tile (K blocks kb = 0..3 at 32-byte
+// descriptor steps, scale columns 4 kb / 8 kb further), issued back to back from one
+// asm block so that no other instruction sits between them.  The first MMA
+// accumulates iff `accumulate`; the other three always do.
+__device__ __forceinline__ void mma_nvfp4_x4(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                             uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.eq.b32 q, %4, %4;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%9], p;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %10, %11, %3, [%6], [%12], q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %13, %14, %3, [%7], [%15], q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %16, %17, %3, [%8], [%18], q;\n\t}" ::"r"(
+          d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfa_tmem + 4), "r"(sfa_tmem + 8),
+      "r"(sfa_tmem + 12), "r"(sfb_tmem), "l"(a + 2), "l"(b + 2), "r"(sfb_tmem + 8), "l"(a + 4), "l"(b + 4),
+      "r"(sfb_tmem + 16), "l"(a + 6), "l"(b + 6), "r"(sfb_tmem + 24)
+      : "memory");
+}
 // Arrives once on `bar` when every tcgen05 operation this thread issued so far is done.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(

@@ -70,6 +70,9 @@ struct GemmArgs {
 };
 svdq_status launch_gemm_w4a4(const GemmArgs& a, cudaStream_t stream);
 
+// Device self-test of the encoder's exact division and reciprocal shortcuts.
+svdq_status selftest_codec(unsigned int* mismatches_out);
+
 // NVFP4 codes + atom-layout scales of a device fp32 [rows, K] matrix.
 svdq_status launch_weight_codec(const float* d_src, int rows, int K, uint8_t* codes, uint8_t* sf,
                                 cudaStream_t stream);

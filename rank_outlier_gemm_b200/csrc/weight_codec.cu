@@ -13,6 +13,9 @@ using namespace dev;
 
 __global__ void weight_codec_kernel(const float* __restrict__ src, int rows, int rows_pad, int K,
                                     uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
+  __shared__ float rcp_tbl[16];
+  if (threadIdx.x < 16) rcp_tbl[threadIdx.x] = rcp_table_entry(static_cast<int>(threadIdx.x));
+  __syncthreads();
   const int q_total = K / 64;
   const long idx = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= static_cast<long>(rows_pad) * q_total) return;
@@ -37,7 +40,7 @@ __global__ void weight_codec_kernel(const float* __restrict__ src, int rows, int
 #pragma unroll
       for (int j = 0; j < 16; ++j) v[j] = 0.0f;
     }
-    const Fp4Group gq = nvfp4_encode16(v);
+    const Fp4Group gq = nvfp4_encode16(v, rcp_tbl);
     w[2 * g] = gq.lo;
     w[2 * g + 1] = gq.hi;
     sc |= gq.scale << (8 * g);
@@ -51,7 +54,42 @@ __global__ void weight_codec_kernel(const float* __restrict__ src, int rows, int
   *reinterpret_cast<uint32_t*>(sf + off) = sc;
 }
 
+// Checks the encoder's exact shortcuts against the IEEE intrinsics: div6_rn for
+// every fp32 mantissa at each exponent in [-100, 12] (block x = exponent), and
+// e4m3_rcp for every positive finite E4M3 byte.  Counts mismatches.
+__global__ void selftest_codec_kernel(unsigned int* mismatches) {
+  __shared__ float rcp_tbl[16];
+  if (threadIdx.x < 16) rcp_tbl[threadIdx.x] = rcp_table_entry(static_cast<int>(threadIdx.x));
+  __syncthreads();
+  const int ex = static_cast<int>(blockIdx.y) - 100;
+  unsigned int bad = 0;
+  for (uint32_t mant = blockIdx.x * blockDim.x + threadIdx.x; mant < (1u << 23); mant += gridDim.x * blockDim.x) {
+    const float x = __uint_as_float((static_cast<uint32_t>(ex + 127) << 23) | mant);
+    bad += __float_as_uint(div6_rn(x)) != __float_as_uint(__fdiv_rn(x, 6.0f));
+  }
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x < 127) {
+    const uint32_t b = threadIdx.x;  // 0..126 (0x7F is NaN)
+    const float want = b ? __frcp_rn(e4m3_to_f32(b)) : 0.0f;
+    bad += __float_as_uint(e4m3_rcp(b, rcp_tbl)) != __float_as_uint(want);
+  }
+  if (bad) atomicAdd(mismatches, bad);
+}
+
 }  // namespace
+
+svdq_status selftest_codec(unsigned int* mismatches_out) {
+  unsigned int* d = nullptr;
+  SVDQ_CUDA_TRY(cudaMalloc(&d, sizeof(unsigned int)));
+  cudaError_t e = cudaMemset(d, 0, sizeof(unsigned int));
+  if (e == cudaSuccess) {
+    selftest_codec_kernel<<<dim3(512, 113), 256>>>(d);
+    e = cudaGetLastError();
+  }
+  if (e == cudaSuccess) e = cudaMemcpy(mismatches_out, d, sizeof(unsigned int), cudaMemcpyDeviceToHost);
+  cudaFree(d);
+  if (e != cudaSuccess) return cuda_fail(e, "codec self-test");
+  return SVDQ_OK;
+}
 
 svdq_status launch_weight_codec(const float* d_src, int rows, int K, uint8_t* codes, uint8_t* sf,
                                 cudaStream_t stream) {

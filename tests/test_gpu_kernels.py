@@ -148,6 +148,13 @@ def test_forward_entry_points_agree():
     np.testing.assert_array_equal(Yh.float().numpy(), Y2)
 
 
+def test_codec_shortcuts_match_ieee():
+    """The encoder's fused division by 6 and its table reciprocal of the E4M3
+    scale equal IEEE fp32 division / reciprocal over their whole domains
+    (checked on the device against the IEEE intrinsics)."""
+    assert G.lib().svdq_selftest_codec() == 0
+
+
 def test_output_only_16_byte_aligned():
     """Y that is 16- but not 32-byte aligned takes the 16-byte store path; the
     values are the same as with an aligned Y (and rows/columns stay in place)."""
