@@ -60,7 +60,12 @@ def peaks():
 # gemm_w4a4_kernel on this workload, from one ncu capture, with the SHA-256 of the
 # kernel source the counters were taken on; counters of another source are stale
 # and not reported.
-K2_TRAFFIC = {"source_sha256": None, "bytes_per_launch": {}}
+K2_TRAFFIC = {
+    "source_sha256": "c33a1cc9f7370360dd404b28c33b271763f949f69845fa91e8d1da98a97dad2b",
+    # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum: read + write per launch
+    "bytes_per_launch": {"attn_out": 14104064 + 11520, "qkv": 25144064 + 32850944,
+                         "mlp_up": 30659328 + 59751168, "mlp_down": 55489536 + 5601792},
+}
 
 
 def k2_traffic_per_launch(names):
