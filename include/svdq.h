@@ -163,9 +163,15 @@ svdq_status svdq_forward(const svdq_weights* w, const void* X_bf16, int M, void*
 
 /*
  * svdq_forward with host input and output: copies X (host, M x K bf16) into
- * the workspace, runs both kernels and copies Y (M x N bf16) back into Y_host,
- * all enqueued on `stream` (no synchronization).  `workspace` is device memory
- * of at least svdq_forward_host_workspace_bytes(w, M) bytes.
+ * the workspace, runs both kernels and copies Y (M x N bf16) back into Y_host.
+ * `workspace` is device memory of at least svdq_forward_host_workspace_bytes(w, M)
+ * bytes.  For M >= 1024 the rows are processed in up to four chunks of a
+ * multiple of 128 rows: uploads and downloads run on two copy streams the
+ * library keeps per device, the kernels on `stream`, so the copies of one
+ * chunk overlap the kernels of its neighbours (X_host and Y_host should be
+ * pinned for the copies to be asynchronous).  Nothing synchronizes: the work
+ * is ordered after what `stream` already holds, and `stream` is ordered after
+ * all of it.  Calls for one device are enqueued one at a time.
  */
 svdq_status svdq_forward_host(const svdq_weights* w, const void* X_host, int M, void* Y_host,
                               void* workspace, size_t workspace_bytes, void* stream);

@@ -249,6 +249,44 @@ svdq_status check_dev_ptr(const void* p, const char* name) {
 
 using namespace svdq;
 
+namespace {
+
+// Copy streams and events of svdq_forward_host, one set per device, created on
+// first use and kept for the life of the process.
+struct HostPipe {
+  static constexpr int kMaxChunks = 4;
+  std::mutex mu;  // one call at a time enqueues on a device's pipe
+  bool ready = false;
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t start = nullptr, done = nullptr;
+  cudaEvent_t loaded[kMaxChunks] = {}, computed[kMaxChunks] = {};
+};
+HostPipe g_host_pipe[64];
+std::mutex g_host_pipe_mu;
+
+svdq_status host_pipe(HostPipe** out) {
+  int dev = 0;
+  SVDQ_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(SVDQ_ERR_UNSUPPORTED_DEVICE, "device index %d", dev);
+  std::lock_guard<std::mutex> lk(g_host_pipe_mu);
+  HostPipe& hp = g_host_pipe[dev];
+  if (!hp.ready) {
+    SVDQ_CUDA_TRY(cudaStreamCreateWithFlags(&hp.in, cudaStreamNonBlocking));
+    SVDQ_CUDA_TRY(cudaStreamCreateWithFlags(&hp.out, cudaStreamNonBlocking));
+    SVDQ_CUDA_TRY(cudaEventCreateWithFlags(&hp.start, cudaEventDisableTiming));
+    SVDQ_CUDA_TRY(cudaEventCreateWithFlags(&hp.done, cudaEventDisableTiming));
+    for (int c = 0; c < HostPipe::kMaxChunks; ++c) {
+      SVDQ_CUDA_TRY(cudaEventCreateWithFlags(&hp.loaded[c], cudaEventDisableTiming));
+      SVDQ_CUDA_TRY(cudaEventCreateWithFlags(&hp.computed[c], cudaEventDisableTiming));
+    }
+    hp.ready = true;
+  }
+  *out = &hp;
+  return SVDQ_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 void svdq_prepare_opts_default(svdq_prepare_opts* o) {
@@ -420,12 +458,44 @@ svdq_status svdq_forward_host(const svdq_weights* w, const void* X_host, int M, 
                 svdq_forward_host_workspace_bytes(w, M));
   const size_t fw = svdq_forward_workspace_bytes(w, M);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint8_t* xq = ws;
+  uint8_t* xsf = xq + up256(svdq_act_codes_bytes(M, w->K));
+  uint8_t* T = xsf + up256(svdq_act_sf_bytes(M, w->K));
   uint8_t* dX = ws + fw;
   uint8_t* dY = dX + up256(static_cast<size_t>(M) * w->K * 2);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  SVDQ_CUDA_TRY(cudaMemcpyAsync(dX, X_host, static_cast<size_t>(M) * w->K * 2, cudaMemcpyHostToDevice, s));
-  SVDQ_TRY(svdq_forward(w, dX, M, dY, ws, fw, stream));
-  SVDQ_CUDA_TRY(cudaMemcpyAsync(Y_host, dY, static_cast<size_t>(M) * w->N * 2, cudaMemcpyDeviceToHost, s));
+  const size_t xrow = static_cast<size_t>(w->K) * 2, yrow = static_cast<size_t>(w->N) * 2;
+  const uint8_t* Xh = static_cast<const uint8_t*>(X_host);
+  uint8_t* Yh = static_cast<uint8_t*>(Y_host);
+
+  // Rows are split into chunks (multiples of 128 rows) so that the upload of
+  // chunk c+1 and the download of chunk c-1 run on their own streams while the
+  // kernels of chunk c run on the caller's stream.  Every chunk owns disjoint
+  // rows of the workspace, so only the per-chunk events order the three streams.
+  const int nch = std::max(1, std::min(HostPipe::kMaxChunks, M / 512));
+  const int rows = round_up((M + nch - 1) / nch, 128);
+  HostPipe* hp = nullptr;
+  SVDQ_TRY(host_pipe(&hp));
+  std::lock_guard<std::mutex> lk(hp->mu);
+  SVDQ_CUDA_TRY(cudaEventRecord(hp->start, s));
+  SVDQ_CUDA_TRY(cudaStreamWaitEvent(hp->in, hp->start, 0));
+  SVDQ_CUDA_TRY(cudaStreamWaitEvent(hp->out, hp->start, 0));
+  for (int c = 0, m0 = 0; m0 < M; ++c, m0 += rows) {
+    const int mc = std::min(rows, M - m0);
+    SVDQ_CUDA_TRY(cudaMemcpyAsync(dX + m0 * xrow, Xh + m0 * xrow, mc * xrow, cudaMemcpyHostToDevice, hp->in));
+    SVDQ_CUDA_TRY(cudaEventRecord(hp->loaded[c], hp->in));
+    SVDQ_CUDA_TRY(cudaStreamWaitEvent(s, hp->loaded[c], 0));
+    uint8_t* Tc = w->r_pad ? T + static_cast<size_t>(m0) * 4 * w->r_pad : nullptr;
+    SVDQ_TRY(svdq_quantize_act_lowrank_down(w, dX + m0 * xrow, mc, xq + static_cast<size_t>(m0) * (w->K / 2),
+                                            xsf + static_cast<size_t>(m0) * (w->K / 16), Tc, stream));
+    SVDQ_TRY(svdq_linear_w4a4(w, xq + static_cast<size_t>(m0) * (w->K / 2),
+                              xsf + static_cast<size_t>(m0) * (w->K / 16), Tc, mc, dY + m0 * yrow, stream));
+    SVDQ_CUDA_TRY(cudaEventRecord(hp->computed[c], s));
+    SVDQ_CUDA_TRY(cudaStreamWaitEvent(hp->out, hp->computed[c], 0));
+    SVDQ_CUDA_TRY(cudaMemcpyAsync(Yh + m0 * yrow, dY + m0 * yrow, mc * yrow, cudaMemcpyDeviceToHost, hp->out));
+  }
+  SVDQ_CUDA_TRY(cudaEventRecord(hp->done, hp->out));
+  SVDQ_CUDA_TRY(cudaStreamWaitEvent(s, hp->done, 0));
   return SVDQ_OK;
 }
 

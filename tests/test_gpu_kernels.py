@@ -148,6 +148,26 @@ def test_forward_entry_points_agree():
     np.testing.assert_array_equal(Yh.float().numpy(), Y2)
 
 
+def test_forward_host_chunked_pipeline():
+    """A host-buffer call large enough to be split into row chunks (two chunks,
+    the second ragged) gives the same output as the device-buffer call."""
+    L = G.lib()
+    t, prep = _case_prep("pixart/mlp_up", 1100)
+    w = G.weights_from_oracle(prep)
+    M = t.X_bits.shape[0]
+    X = G.to_dev_bf16(t.X_bits)
+    Y = torch.empty((M, w.info["N"]), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(L.svdq_forward_workspace_bytes(w, M), dtype=torch.uint8, device="cuda")
+    L.svdq_forward(w, X, Y, ws)
+    Xh = torch.from_numpy(t.X_bits.view(np.int16).copy()).view(torch.bfloat16).pin_memory()
+    Yh = torch.full((M, w.info["N"]), float("nan"), dtype=torch.bfloat16).pin_memory()
+    wsh = torch.empty(L.svdq_forward_host_workspace_bytes(w, M), dtype=torch.uint8, device="cuda")
+    L.svdq_forward_host(w, Xh, Yh, wsh)
+    torch.cuda.synchronize()
+    assert L.svdq_check_device_errors() == 0
+    np.testing.assert_array_equal(Yh.float().numpy(), Y.float().cpu().numpy())
+
+
 def test_codec_shortcuts_match_ieee():
     """The encoder's fused division by 6 and its table reciprocal of the E4M3
     scale equal IEEE fp32 division / reciprocal over their whole domains
