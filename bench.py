@@ -137,6 +137,101 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(sm)}
 
 
+# ------------------------------------------------------------------ extras
+def _time_ms(torch, stream, fn, reps):
+    for _ in range(3):
+        fn()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record(stream)
+    for _ in range(reps):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps
+
+
+def unfused_overhead(L, torch, layers, stream, ms0, reps):
+    """The low-rank branch run unfused (SVDQuant §4.3, Fig. 6: the naive
+    implementation): both kernels at rank 0, then T = X L1' and Y += T L2 as two
+    separate cuBLAS bf16 GEMMs that re-read X and re-write Y.  Returns its step
+    time over the rank-0 step's, minus one."""
+    extra = []
+    for l in layers:
+        ex = L.svdq_weights_export(l["w"])
+        dev = l["X"].device
+        L1p = torch.from_numpy(ex["L1p"].view(np.int16).copy()).view(torch.bfloat16).to(dev)
+        L2 = torch.from_numpy(ex["L2"].view(np.int16).copy()).view(torch.bfloat16).to(dev)
+        extra.append((L1p, L2))
+
+    def step_unfused():
+        for l, (L1p, L2) in zip(layers, extra):
+            xq, xsf, _ = l["bufs"]
+            L.svdq_quantize_act_lowrank_down(l["w0"], l["X"], xq, xsf, None)
+            L.svdq_linear_w4a4(l["w0"], xq, xsf, None, l["case"].M, l["Y"])
+            T = l["X"] @ L1p
+            l["Y"].addmm_(T, L2)
+
+    return _time_ms(torch, stream, step_unfused, reps) / ms0 - 1.0
+
+
+def rank_sweep(L, torch, layers, dev, stream, reps=50):
+    """Layer time (both kernels) of the largest step layer at ranks 0, 16, 32,
+    32 + a rank-16 LoRA attached without re-quantization, and 64; the
+    per-rank overhead is relative to rank 0 (SVDQuant App. E.5 trade-off)."""
+    l = max(layers, key=lambda z: z["case"].flops)
+    c = l["case"]
+    t = make_layer_inputs(c)
+    out = {"layer": f"{c.label} M={c.M} K={c.K} N={c.N}", "us": {}, "overhead_vs_rank0": {}}
+    handles = {"0": l["w0"], "32": l["w"]}
+    for r in (16, 64):
+        handles[str(r)] = L.svdq_prepare_weights(t.W_bits, t.act_absmax, t.bias_bits, rank=r)
+    wl = L.svdq_prepare_weights(t.W_bits, t.act_absmax, t.bias_bits, rank=32)
+    g = np.random.default_rng(7)
+    A = (g.standard_normal((c.K, 16)) * 0.01).astype(np.float32)
+    B = (g.standard_normal((16, c.N)) * 0.01).astype(np.float32)
+    to_bits = lambda a: torch.from_numpy(a).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    L.svdq_attach_lora(wl, to_bits(A), to_bits(B), 1.0)
+    handles["32+lora16"] = wl
+    for key, w in handles.items():
+        xq, xsf, T = L.act_buffers(w, c.M, dev)
+
+        def one():
+            L.svdq_quantize_act_lowrank_down(w, l["X"], xq, xsf, T)
+            L.svdq_linear_w4a4(w, xq, xsf, T, c.M, l["Y"])
+
+        out["us"][key] = 1e3 * _time_ms(torch, stream, one, reps)
+    for key, us in out["us"].items():
+        out["overhead_vs_rank0"][key] = us / out["us"]["0"] - 1.0
+    return out
+
+
+def small_m(L, torch, dev, stream, reps=100):
+    """The small-M + LoRA configuration (K = 3072, N in {3072, 12288}, M in {1, 16,
+    256}, rank 32 + a rank-16 LoRA): layer time (both kernels) and the fraction of
+    its HBM floor (weight codes + scales + low-rank factors + X + Y at the measured
+    copy bandwidth)."""
+    hbm = peaks()["hbm"] * 1e9
+    out = {}
+    for c in config_cases("small_m_lora"):
+        t = make_layer_inputs(c)
+        w = L.svdq_prepare_weights(t.W_bits, t.act_absmax, t.bias_bits, rank=c.rank)
+        L.svdq_attach_lora(w, t.lora_A_bits, t.lora_B_bits, 1.0)
+        X = torch.from_numpy(t.X_bits.view(np.int16).copy()).view(torch.bfloat16).to(dev)
+        Y = torch.empty((c.M, c.N), dtype=torch.bfloat16, device=dev)
+        xq, xsf, T = L.act_buffers(w, c.M, dev)
+
+        def one():
+            L.svdq_quantize_act_lowrank_down(w, X, xq, xsf, T)
+            L.svdq_linear_w4a4(w, xq, xsf, T, c.M, Y)
+
+        us = 1e3 * _time_ms(torch, stream, one, reps)
+        r = c.rank + c.lora_rank
+        floor = (c.N * c.K * (0.5 + 1 / 16) + 2 * r * (c.K + c.N) + 2 * c.M * (c.K + c.N)) / hbm * 1e6
+        out[c.name] = {"us": us, "hbm_floor_us": floor, "frac": floor / us}
+    return out
+
+
 # ------------------------------------------------------------------ ours
 def run_ours(args):
     import torch
@@ -228,6 +323,7 @@ def run_ours(args):
 
     # low-rank overhead: the same kernels at rank 0 (extras)
     overhead = None
+    unfused = sweep = small = None
     if args.extras:
         def step0():
             for l in layers:
@@ -246,6 +342,10 @@ def run_ours(args):
         torch.cuda.synchronize()
         ms0 = a.elapsed_time(b) / n0
         overhead = ms_step / ms0 - 1.0
+        if rank == 0:
+            unfused = unfused_overhead(L, torch, layers, stream, ms0, n0)
+            sweep = rank_sweep(L, torch, layers, dev, stream)
+            small = small_m(L, torch, dev, stream)
 
     # end to end through the public host-buffer call: H2D of X, both kernels, D2H of Y
     e2e = None
@@ -294,6 +394,9 @@ def run_ours(args):
                          "kernel": "gemm_w4a4_kernel", "peak_source": peak_src,
                          "frac_of_datasheet_9pf": achieved / 9000.0},
             "lowrank_overhead_vs_rank0": overhead,
+            "unfused_lowrank_overhead_vs_rank0": unfused,
+            "rank_sweep": sweep,
+            "small_m_lora": small,
             "gpu_launches": 2 * nl * args.steps,
             "e2e": e2e,
         }
