@@ -145,12 +145,8 @@ __global__ void __launch_bounds__(kThreads, 2) act_quant_lowrank_kernel(
         const uint32_t ph = (i / kStages) & 1;
         if (!wait_bounded(&sh->full[s], ph, wc)) break;
         tc_fence_after();
-        const uint32_t xa = smem_u32(xs + s * kXTile);
-        const uint32_t la = smem_u32(l1s + s * p.l1_tile);
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          mma_bf16(tmem, desc_kmajor_sw128(xa + 32 * k), desc_kmajor_sw128(la + 32 * k), idesc,
-                   (i | k) != 0);
+        mma_bf16_x4(tmem, desc_kmajor_sw128(smem_u32(xs + s * kXTile)),
+                    desc_kmajor_sw128(smem_u32(l1s + s * p.l1_tile)), idesc, i != 0);
         mma_commit(&sh->empty[s]);
       }
       mma_commit(&sh->tfull);

@@ -238,12 +238,6 @@ svdq_status check_dev_ptr(const void* p, const char* name) {
   return SVDQ_OK;
 }
 
-#define SVDQ_TRY(expr)                 \
-  do {                                 \
-    svdq_status _s = (expr);           \
-    if (_s != SVDQ_OK) return _s;      \
-  } while (0)
-
 }  // namespace
 }  // namespace svdq
 

@@ -225,6 +225,24 @@ __device__ __forceinline__ void mma_nvfp4(uint32_t d_tmem, uint64_t a, uint64_t 
       "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
       : "memory");
 }
+// Four kind::f16 MMAs (bf16, K = 16 each) over one 64-element K block: A and B
+// descriptors advance 32 bytes per MMA; the first accumulates iff `accumulate`.
+// One asm block keeps other instructions from sitting between them.
+__device__ __forceinline__ void mma_bf16_x4(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.eq.b32 q, %4, %4;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %5, %6, %3, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %7, %8, %3, q;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %9, %10, %3, q;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "l"(a + 2), "l"(b + 2), "l"(a + 4), "l"(b + 4), "l"(a + 6),
+      "l"(b + 6)
+      : "memory");
+}
+
 // Four block-scaled MMAs over one 256-wide K tile (K blocks kb = 0..3 at 32-byte
 // descriptor steps, scale columns 4 kb / 8 kb further), issued back to back from one
 // asm block so that no other instruction sits between them.  The first MMA

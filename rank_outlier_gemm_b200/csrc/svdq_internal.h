@@ -23,6 +23,13 @@ svdq_status cuda_fail(cudaError_t e, const char* what);
     if (_e != cudaSuccess) return ::svdq::cuda_fail(_e, #expr); \
   } while (0)
 
+// Returns the status of `expr` from the enclosing function unless it is SVDQ_OK.
+#define SVDQ_TRY(expr)                 \
+  do {                                 \
+    svdq_status _s = (expr);           \
+    if (_s != SVDQ_OK) return _s;      \
+  } while (0)
+
 // Device error word of the current device (lazily allocated, zeroed).
 int* device_error_word();
 uint64_t wait_limit_ns();

@@ -53,6 +53,29 @@ def test_activation_codes_bitexact(M, K):
     G.check_codes(xq, xsf, Xf, inv_lam)
 
 
+@pytest.mark.parametrize("M,K", [(4600, 1152), (8000, 640)])
+def test_large_M_layer(M, K):
+    """Large M (ragged last row block at M = 4600; K = 640 is a ragged number of
+    256-wide GEMM K tiles): codes and scales bit-exact, T within the fp32
+    accumulation bound, and the whole layer within the output tolerance on
+    rows from the start, middle and end."""
+    rng = np.random.default_rng(M + K)
+    X = rng.normal(0, 1, (M, K)).astype(np.float32)
+    X[:, rng.choice(K, 5, replace=False)] *= 30
+    X[7, :64] = 0.0
+    Xb = f32_to_bf16_bits(X)
+    Xf = OF.bf16_bits_to_f64(Xb).astype(np.float32)
+    W = rng.normal(0, 0.02, (64, K)).astype(np.float32)
+    bias = rng.normal(0, 0.01, 64).astype(np.float32)
+    prep = OS.prepare(W, np.abs(Xf).max(axis=0), bias, 32)
+    w = G.weights_from_oracle(prep)
+    Y, (xq, xsf, T) = G.run_layer(w, Xb)
+    G.check_codes(xq, xsf, Xf, prep.inv_lam)
+    G.check_T(T, Xf, prep)
+    rows = np.r_[0:40, M // 2 : M // 2 + 40, M - 40 : M]
+    G.check_Y(Y[rows], OS.linear(prep, Xf, rows=rows))
+
+
 def test_weight_codes_and_factor_bitexact():
     t, prep = _case_prep("pixart/attn_qkv_out", 128)
     w = G.weights_from_oracle(prep)
