@@ -232,6 +232,22 @@ def small_m(L, torch, dev, stream, reps=100):
     return out
 
 
+def refinement(L, iters=4):
+    """NEXT-2 (SVDQuant §4.2, iterative refinement of the split): residual
+    quantization error of each split tried and the host preparation time,
+    plain vs refined, on one SDXL attention layer."""
+    c = config_cases("sdxl")[0]
+    t = make_layer_inputs(c)
+    out = {"layer": f"{c.label} N={c.N} K={c.K} rank={c.rank}"}
+    for it in (1, iters):
+        t0 = time.time()
+        w = L.svdq_prepare_weights(t.W_bits, t.act_absmax, t.bias_bits, rank=c.rank, refine_iters=it)
+        out[f"iters{it}"] = {"errors": L.svdq_weights_refine_errors(w), "prepare_s": time.time() - t0}
+    e1, e4 = out["iters1"]["errors"][0], min(out[f"iters{iters}"]["errors"])
+    out["error_reduction"] = 1.0 - e4 / e1
+    return out
+
+
 # ------------------------------------------------------------------ ours
 def run_ours(args):
     import torch
@@ -323,7 +339,7 @@ def run_ours(args):
 
     # low-rank overhead: the same kernels at rank 0 (extras)
     overhead = None
-    unfused = sweep = small = None
+    unfused = sweep = small = refine = None
     if args.extras:
         def step0():
             for l in layers:
@@ -346,6 +362,7 @@ def run_ours(args):
             unfused = unfused_overhead(L, torch, layers, stream, ms0, n0)
             sweep = rank_sweep(L, torch, layers, dev, stream)
             small = small_m(L, torch, dev, stream)
+            refine = refinement(L)
 
     # end to end through the public host-buffer call: H2D of X, both kernels, D2H of Y
     e2e = None
@@ -397,6 +414,7 @@ def run_ours(args):
             "unfused_lowrank_overhead_vs_rank0": unfused,
             "rank_sweep": sweep,
             "small_m_lora": small,
+            "refinement": refine,
             "gpu_launches": 2 * nl * args.steps,
             "e2e": e2e,
         }

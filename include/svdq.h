@@ -67,6 +67,7 @@ typedef struct {
   int oversample;     /* extra columns of the random subspace; default 16 */
   uint64_t seed;      /* seed of the random starting subspace; default 0 */
   int keep_residual;  /* nonzero: keep a host copy of R/alpha_w for export */
+  int refine_iters;   /* splits tried (§4.2 refinement, see svdq_prepare_weights); default 1 */
 } svdq_prepare_opts;
 
 /* Fills *opts with the defaults above. */
@@ -81,6 +82,12 @@ void svdq_prepare_opts_default(svdq_prepare_opts* opts);
  * R = W_hat - (diag(1/inv_lam) L1' L2)^T, the power-of-two factor
  * alpha_w = 2^ceil(log2(max|R| / 2688)), and the NVFP4 codes of R/alpha_w
  * (computed on the device).
+ * With opts->refine_iters = t > 1 the split is refined (§4.2: the
+ * decomposition can be refined over several iterations; the update is a
+ * reading): with Q(R) = alpha_w times the NVFP4 round trip of R/alpha_w,
+ * L_{i+1} = SVD_r(W_hat - Q(W_hat - L_i)) for i < t, and the split whose
+ * residual quantization error ||R - Q(R)||_F is smallest is kept
+ * (svdq_weights_refine_errors reports the errors).
  *   W_bf16      host, N x K bf16 (out x in)
  *   act_absmax  host, K floats: per-input-channel max |x| over calibration data
  *   bias_bf16   host, N bf16, or NULL for no bias
@@ -92,6 +99,15 @@ svdq_status svdq_prepare_weights(const uint16_t* W_bf16, const float* act_absmax
                                  const uint16_t* bias_bf16, int N, int K,
                                  const svdq_prepare_opts* opts, void* stream,
                                  svdq_weights** out);
+
+/*
+ * The residual quantization error ||R - Q(R)||_F (Frobenius, float64, in the
+ * smoothed-weight space) of each split svdq_prepare_weights tried, in order:
+ * one value without refinement, refine_iters values with it (the kept split
+ * has the smallest); 0 values for handles made by svdq_weights_from_factors.
+ * Writes min(count, max_count) values to `errors` (host) and the count to *count.
+ */
+svdq_status svdq_weights_refine_errors(const svdq_weights* w, double* errors, int max_count, int* count);
 
 /*
  * Builds a handle from a given split (the second half of

@@ -28,6 +28,13 @@ Steps and where they come from:
      (exact).  It keeps the weight block scales out of the E4M3 subnormals;
      a power of two adds no rounding.
   4. NVFP4 codec (see ``codec.py``) on R' rows and on X_hat = fp32(x * inv_lam).
+  4b. Optional refinement (§4.2: the decomposition "can be refined over several
+     iterations"; the pages give no formula).  Reading: with Q(R) the weight
+     quantization as the runtime sees it (alpha_w times the dequantized codes of
+     R/alpha_w, App. A.2's Q(R) = s_R Q_R), iterate
+     L_{t+1} = SVD_r(W_hat - Q(W_hat - L_t)) starting from the plain split, and
+     keep the split whose residual quantization error ||R - Q(R)||_F is
+     smallest (R computed from the stored 16-bit factors as in step 2).
   5. Output in float64 with no intermediate rounding:
      Y = alpha_w deq(Qx) deq(Qw)^T + (X L1') L2b + b.
   6. LoRA (§2 and §5.2 Fig. 9: off-the-shelf LoRAs are absorbed into the
@@ -106,6 +113,7 @@ class Prepared:
     w_scales: np.ndarray     # uint8 [N, K/16]
     bias: np.ndarray         # float64 [N]
     sigma: Optional[np.ndarray] = None       # singular values of W_hat
+    refine_errors: Optional[list] = None     # ||R - Q(R)||_F of each split tried (step 4b)
     lora_B_exact: Optional[np.ndarray] = None  # float64 scale*B rows appended to L2b
     lora_rank: int = 0
 
@@ -128,14 +136,33 @@ def prepare_from_factors(W_hat, inv_lam, L1p, L2b, bias, lam=None, sigma=None) -
                     L1p, L2b, R, aw, Rp, codes, scales, b, sigma)
 
 
-def prepare(W, act_absmax, bias, rank: int, alpha: float = 0.5) -> Prepared:
-    """Smoothing, SVD split, residual quantization (steps 1-4 for the weights)."""
+def fake_quantize_weights(R) -> np.ndarray:
+    """Q(R) = alpha_w * dequantized NVFP4 codes of R / alpha_w, float64 (step 4b)."""
+    R = np.asarray(R, np.float32)
+    aw = weight_factor(R)
+    codes, scales = quantize_groups((R.astype(np.float64) / aw).astype(np.float32))
+    return dequantize_groups(codes, scales) * aw
+
+
+def prepare(W, act_absmax, bias, rank: int, alpha: float = 0.5, iters: int = 1) -> Prepared:
+    """Smoothing, SVD split, residual quantization (steps 1-4 for the weights);
+    ``iters`` > 1 refines the split (step 4b) and keeps the best of ``iters``."""
     lam, inv_lam = smoothing_factors(act_absmax, W, alpha)
     W_hat = smooth_weight(W, inv_lam)
-    L1, L2, s = svd_split(W_hat, rank)
-    L1p = round_bf16(L1 * inv_lam.astype(np.float64)[:, None])
-    L2b = round_bf16(L2)
-    return prepare_from_factors(W_hat, inv_lam, L1p, L2b, bias, lam=lam, sigma=s)
+    inv64 = inv_lam.astype(np.float64)[:, None]
+    A = W_hat
+    best, errors = None, []
+    for _ in range(max(1, iters)):
+        L1, L2, s = svd_split(A, rank)
+        prep = prepare_from_factors(W_hat, inv_lam, round_bf16(L1 * inv64), round_bf16(L2), bias, lam=lam,
+                                    sigma=s if best is None else best.sigma)
+        Q = fake_quantize_weights(prep.R)
+        errors.append(float(np.linalg.norm(prep.R.astype(np.float64) - Q)))
+        if best is None or errors[-1] < min(errors[:-1]):
+            best = prep
+        A = W_hat - Q
+    best.refine_errors = errors
+    return best
 
 
 def smooth_activations(X, inv_lam) -> np.ndarray:

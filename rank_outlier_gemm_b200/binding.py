@@ -32,7 +32,8 @@ class SvdqError(RuntimeError):
 
 class PrepareOpts(ctypes.Structure):
     _fields_ = [("alpha", ctypes.c_float), ("rank", ctypes.c_int), ("power_iters", ctypes.c_int),
-                ("oversample", ctypes.c_int), ("seed", ctypes.c_uint64), ("keep_residual", ctypes.c_int)]
+                ("oversample", ctypes.c_int), ("seed", ctypes.c_uint64), ("keep_residual", ctypes.c_int),
+                ("refine_iters", ctypes.c_int)]
 
 
 _vp, _i, _sz, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
@@ -58,6 +59,7 @@ _SIGS = {
     "svdq_set_wait_limit_ns": (None, [ctypes.c_uint64]),
     "svdq_check_device_errors": (_i, [_vp]),
     "svdq_selftest_codec": (_i, [ctypes.POINTER(ctypes.c_uint)]),
+    "svdq_weights_refine_errors": (_i, [_vp, ctypes.POINTER(ctypes.c_double), _i, ctypes.POINTER(_i)]),
     "svdq_debug_launch_stalled_act": (_i, [_vp, _vp, _i, _vp, _vp, _vp, _vp]),
     "svdq_last_error": (ctypes.c_char_p, []),
     "svdq_version": (ctypes.c_char_p, []),
@@ -146,7 +148,7 @@ def svdq_prepare_opts_default() -> PrepareOpts:
 
 def svdq_prepare_weights(W_bf16, act_absmax, bias_bf16=None, rank: int = 32, alpha: float = 0.5,
                          power_iters: int = 4, oversample: int = 16, seed: int = 0,
-                         keep_residual: bool = False, stream=None) -> Weights:
+                         keep_residual: bool = False, refine_iters: int = 1, stream=None) -> Weights:
     Wp, Wk = _host(W_bf16, np.uint16)
     N, K = Wk.shape
     ap, ak = _host(act_absmax, np.float32)
@@ -154,6 +156,7 @@ def svdq_prepare_weights(W_bf16, act_absmax, bias_bf16=None, rank: int = 32, alp
     o = svdq_prepare_opts_default()
     o.alpha, o.rank, o.power_iters, o.oversample, o.seed = alpha, rank, power_iters, oversample, seed
     o.keep_residual = int(keep_residual)
+    o.refine_iters = int(refine_iters)
     h = _vp()
     _check(_lib.svdq_prepare_weights(Wp, ap, bp, N, K, ctypes.byref(o), _stream(stream), ctypes.byref(h)),
            "svdq_prepare_weights")
@@ -259,6 +262,15 @@ def svdq_weights_export(w: Weights, residual: bool = False) -> dict:
 
 def svdq_set_wait_limit_ns(ns: int) -> None:
     _lib.svdq_set_wait_limit_ns(int(ns))
+
+
+def svdq_weights_refine_errors(w: Weights) -> list:
+    """Residual quantization error of each split prepare tried (the kept one is the smallest)."""
+    n = ctypes.c_int(0)
+    _check(_lib.svdq_weights_refine_errors(w.handle, None, 0, ctypes.byref(n)), "svdq_weights_refine_errors")
+    buf = (ctypes.c_double * max(1, n.value))()
+    _check(_lib.svdq_weights_refine_errors(w.handle, buf, n.value, ctypes.byref(n)), "svdq_weights_refine_errors")
+    return [float(buf[i]) for i in range(n.value)]
 
 
 def svdq_selftest_codec() -> int:

@@ -291,6 +291,7 @@ void svdq_prepare_opts_default(svdq_prepare_opts* o) {
   o->oversample = 16;
   o->seed = 0;
   o->keep_residual = 0;
+  o->refine_iters = 1;
 }
 
 svdq_status svdq_prepare_weights(const uint16_t* W_bf16, const float* act_absmax, const uint16_t* bias_bf16,
@@ -306,6 +307,8 @@ svdq_status svdq_prepare_weights(const uint16_t* W_bf16, const float* act_absmax
   if (o.rank < 0 || o.rank > 128 || o.rank > std::min(N, K))
     return fail(SVDQ_ERR_INVALID_ARG, "rank=%d must be in [0, min(128, N, K)]", o.rank);
   if (!(o.alpha >= 0.0f && o.alpha <= 1.0f)) return fail(SVDQ_ERR_INVALID_ARG, "alpha must be in [0, 1]");
+  if (o.refine_iters < 1 || o.refine_iters > 64)
+    return fail(SVDQ_ERR_INVALID_ARG, "refine_iters=%d must be in [1, 64]", o.refine_iters);
   for (int k = 0; k < K; ++k)
     if (!std::isfinite(act_absmax[k]) || act_absmax[k] < 0)
       return fail(SVDQ_ERR_INVALID_ARG, "act_absmax[%d] is negative or not finite", k);
@@ -317,9 +320,19 @@ svdq_status svdq_prepare_weights(const uint16_t* W_bf16, const float* act_absmax
     bias.resize(N);
     for (int n = 0; n < N; ++n) bias[n] = bf16_to_f32(bias_bf16[n]);
   }
-  return build_handle(N, K, o.rank, hs.inv_lam.data(), hs.L1p.data(), hs.L2.data(), hs.R.data(),
-                      bias_bf16 ? bias.data() : nullptr, o.keep_residual, static_cast<cudaStream_t>(stream),
-                      out);
+  SVDQ_TRY(build_handle(N, K, o.rank, hs.inv_lam.data(), hs.L1p.data(), hs.L2.data(), hs.R.data(),
+                        bias_bf16 ? bias.data() : nullptr, o.keep_residual, static_cast<cudaStream_t>(stream),
+                        out));
+  (*out)->refine_err = hs.refine_err;
+  return SVDQ_OK;
+}
+
+svdq_status svdq_weights_refine_errors(const svdq_weights* w, double* errors, int max_count, int* count) {
+  if (!w || !count) return fail(SVDQ_ERR_INVALID_ARG, "null weights handle or count");
+  if (max_count > 0 && !errors) return fail(SVDQ_ERR_INVALID_ARG, "errors is null");
+  *count = static_cast<int>(w->refine_err.size());
+  for (int i = 0; i < std::min(*count, max_count); ++i) errors[i] = w->refine_err[i];
+  return SVDQ_OK;
 }
 
 svdq_status svdq_weights_from_factors(int N, int K, int rank, const float* inv_lam, const uint16_t* L1p_bf16,

@@ -14,6 +14,10 @@
 //  * factors: L1 = U_r S_r (K x r), L2 = V_r^T (r x N); stored as
 //    L1' = bf16(diag(inv_lam) L1) and L2b = bf16(L2); the residual absorbs the
 //    factor rounding: R = W_hat - (diag(1/inv_lam) L1' L2b)^T.
+//  * refinement (§4.2: the split can be refined over several iterations; the
+//    formula is a reading): with Q(R) = alpha_w * (R / alpha_w quantized to
+//    NVFP4 and dequantized), L_{t+1} = SVD_r(W_hat - Q(W_hat - L_t)); the split
+//    with the smallest ||R - Q(R)||_F among the iterations tried is kept.
 #include <algorithm>
 #include <cmath>
 #include <cstring>
@@ -184,6 +188,141 @@ void jacobi_eigen(std::vector<double> G, int n, std::vector<double>& d, std::vec
   E.swap(Es);
 }
 
+// Top-r split of A (N x K) by randomized subspace iteration, 16-bit factors
+// (the smoothing multipliers folded into L1'), and the residual of W_hat that
+// the stored factors leave, R = W_hat - (diag(1/inv_lam) L1' L2b)^T in fp32.
+void split_round_residual(const std::vector<double>& Wh, const std::vector<double>& A, int N, int K,
+                          const svdq_prepare_opts& o, const std::vector<float>& inv_lam, std::vector<uint16_t>* L1p_out,
+                          std::vector<uint16_t>* L2_out, std::vector<float>* R_out) {
+  const int r = o.rank;
+  (*L1p_out).assign(static_cast<size_t>(K) * r, 0);
+  (*L2_out).assign(static_cast<size_t>(r) * N, 0);
+  std::vector<double> L1s(static_cast<size_t>(K) * r, 0.0), L2d(static_cast<size_t>(r) * N, 0.0);
+  if (r > 0) {
+    // ---- randomized subspace iteration
+    const int l = std::min(r + std::max(0, o.oversample), std::min(N, K));
+    std::mt19937_64 gen(o.seed);
+    std::normal_distribution<double> nd(0.0, 1.0);
+    std::vector<double> Om(static_cast<size_t>(K) * l);
+    for (auto& v : Om) v = nd(gen);
+    std::vector<double> Y, Z, Q;
+    mul_a_x(A, N, K, Om, l, Y);
+    orthonormalize(Y, N, l);
+    for (int it = 0; it < std::max(0, o.power_iters); ++it) {
+      mul_at_q(A, N, K, Y, l, Z);
+      orthonormalize(Z, K, l);
+      mul_a_x(A, N, K, Z, l, Y);
+      orthonormalize(Y, N, l);
+    }
+    Q.swap(Y);                       // N x l, orthonormal columns
+    mul_at_q(A, N, K, Q, l, Z);     // Z = A^T Q = B^T  (K x l)
+    // ---- Rayleigh-Ritz: eigen-decomposition of B B^T = Z^T Z (l x l)
+    std::vector<double> G(static_cast<size_t>(l) * l, 0.0);
+    for (int a = 0; a < l; ++a)
+      for (int b = a; b < l; ++b) {
+        double s = 0.0;
+        for (int k = 0; k < K; ++k) s += Z[static_cast<size_t>(k) * l + a] * Z[static_cast<size_t>(k) * l + b];
+        G[static_cast<size_t>(a) * l + b] = G[static_cast<size_t>(b) * l + a] = s;
+      }
+    std::vector<double> d, E;
+    jacobi_eigen(G, l, d, E);
+    // L2 = (Q E_r)^T, L1 = B^T E_r = Z E_r
+    for (int i = 0; i < r; ++i) {
+      for (int n = 0; n < N; ++n) {
+        double s = 0.0;
+        for (int a = 0; a < l; ++a) s += Q[static_cast<size_t>(n) * l + a] * E[static_cast<size_t>(a) * l + i];
+        L2d[static_cast<size_t>(i) * N + n] = s;
+      }
+      for (int k = 0; k < K; ++k) {
+        double s = 0.0;
+        for (int a = 0; a < l; ++a) s += Z[static_cast<size_t>(k) * l + a] * E[static_cast<size_t>(a) * l + i];
+        L1s[static_cast<size_t>(k) * r + i] = s;
+      }
+    }
+    // ---- 16-bit factors; the residual uses them as the runtime does
+    for (int k = 0; k < K; ++k)
+      for (int i = 0; i < r; ++i) {
+        const double v = static_cast<double>(inv_lam[k]) * L1s[static_cast<size_t>(k) * r + i];
+        const uint16_t b = f32_to_bf16_rne(static_cast<float>(v));
+        (*L1p_out)[static_cast<size_t>(k) * r + i] = b;
+        L1s[static_cast<size_t>(k) * r + i] = static_cast<double>(bf16_to_f32(b)) / static_cast<double>(inv_lam[k]);
+      }
+    for (size_t i = 0; i < L2d.size(); ++i) {
+      const uint16_t b = f32_to_bf16_rne(static_cast<float>(L2d[i]));
+      (*L2_out)[i] = b;
+      L2d[i] = bf16_to_f32(b);
+    }
+  }
+  (*R_out).resize(static_cast<size_t>(N) * K);
+  parallel_for(N, [&](long b, long e) {
+    std::vector<double> l2n(std::max(r, 1));
+    for (long n = b; n < e; ++n) {
+      for (int i = 0; i < r; ++i) l2n[i] = L2d[static_cast<size_t>(i) * N + n];
+      for (int k = 0; k < K; ++k) {
+        double low = 0.0;
+        const double* l1 = &L1s[static_cast<size_t>(k) * r];
+        for (int i = 0; i < r; ++i) low += l1[i] * l2n[i];
+        (*R_out)[static_cast<size_t>(n) * K + k] = static_cast<float>(Wh[static_cast<size_t>(n) * K + k] - low);
+      }
+    }
+  });
+}
+
+// NVFP4 round trip of one fp32 value set as the runtime sees it:
+// E4M3 (round to nearest even, saturating) of a non-negative x, as a value.
+double e4m3_rne_sat(double x) {
+  if (x >= 448.0) return 448.0;
+  if (x < 0.015625) return std::nearbyint(x * 512.0) / 512.0;  // subnormals: steps of 2^-9
+  int ex = 0;
+  std::frexp(x, &ex);                                             // x = f 2^ex, f in [0.5, 1)
+  const double step = std::ldexp(1.0, ex - 4);                   // 3 mantissa bits
+  return std::nearbyint(x / step) * step;
+}
+// E2M1 (round to nearest even on {0, .5, 1, 1.5, 2, 3, 4, 6}, saturating), as a value.
+double e2m1_rne_sat(double v) {
+  const double a = std::fabs(v);
+  double q;
+  if (a >= 6.0) q = 6.0;
+  else if (a < 2.0) q = std::nearbyint(a * 2.0) / 2.0;
+  else if (a < 4.0) q = std::nearbyint(a);
+  else q = std::nearbyint(a / 2.0) * 2.0;
+  return v < 0 ? -q : q;
+}
+
+// ||R - Q(R)||_F with Q(R) = alpha_w * NVFP4 round trip of R / alpha_w (groups of
+// 16 along K: s = E4M3(fp32(amax / 6)), codes E2M1(fp32(v * fp32(1 / s))));
+// writes Q(R) (float64, N x K) to *Q if given.
+double fake_quant_error(const std::vector<float>& R, int N, int K, std::vector<double>* Q) {
+  const float aw = weight_factor(R.data(), R.size());
+  if (Q) Q->assign(R.size(), 0.0);
+  std::vector<double> part(static_cast<size_t>(N), 0.0);
+  parallel_for(N, [&](long b, long e) {
+    for (long n = b; n < e; ++n) {
+      double acc = 0.0;
+      for (int g = 0; g < K; g += 16) {
+        const float* row = &R[static_cast<size_t>(n) * K + g];
+        float v[16], amax = 0.0f;
+        for (int i = 0; i < 16; ++i) {
+          v[i] = row[i] / aw;  // exact: aw is a power of two
+          amax = std::max(amax, std::fabs(v[i]));
+        }
+        const double s = e4m3_rne_sat(static_cast<double>(amax / 6.0f));
+        const float rs = s > 0.0 ? 1.0f / static_cast<float>(s) : 0.0f;
+        for (int i = 0; i < 16; ++i) {
+          const double deq = s > 0.0 ? e2m1_rne_sat(static_cast<double>(v[i] * rs)) * s * aw : 0.0;
+          const double d = static_cast<double>(row[i]) - deq;
+          acc += d * d;
+          if (Q) (*Q)[static_cast<size_t>(n) * K + g + i] = deq;
+        }
+      }
+      part[n] = acc;
+    }
+  });
+  double tot = 0.0;
+  for (double x : part) tot += x;
+  return std::sqrt(tot);
+}
+
 }  // namespace
 
 svdq_status host_prepare_split(const uint16_t* W_bf16, const float* act_absmax, int N, int K,
@@ -211,77 +350,26 @@ svdq_status host_prepare_split(const uint16_t* W_bf16, const float* act_absmax, 
             static_cast<double>(out->inv_lam[k]);
   });
 
-  out->L1p.assign(static_cast<size_t>(K) * r, 0);
-  out->L2.assign(static_cast<size_t>(r) * N, 0);
-  std::vector<double> L1s(static_cast<size_t>(K) * r, 0.0), L2d(static_cast<size_t>(r) * N, 0.0);
-  if (r > 0) {
-    // ---- randomized subspace iteration
-    const int l = std::min(r + std::max(0, o.oversample), std::min(N, K));
-    std::mt19937_64 gen(o.seed);
-    std::normal_distribution<double> nd(0.0, 1.0);
-    std::vector<double> Om(static_cast<size_t>(K) * l);
-    for (auto& v : Om) v = nd(gen);
-    std::vector<double> Y, Z, Q;
-    mul_a_x(Wh, N, K, Om, l, Y);
-    orthonormalize(Y, N, l);
-    for (int it = 0; it < std::max(0, o.power_iters); ++it) {
-      mul_at_q(Wh, N, K, Y, l, Z);
-      orthonormalize(Z, K, l);
-      mul_a_x(Wh, N, K, Z, l, Y);
-      orthonormalize(Y, N, l);
+  const int iters = std::max(1, o.refine_iters);
+  std::vector<double> A = Wh;  // matrix whose top-r split is taken (W_hat, then W_hat - Q(R_t))
+  std::vector<double> Q;
+  out->refine_err.clear();
+  for (int t = 0; t < iters; ++t) {
+    std::vector<uint16_t> L1p, L2;
+    std::vector<float> R;
+    split_round_residual(Wh, A, N, K, o, out->inv_lam, &L1p, &L2, &R);
+    const double err = fake_quant_error(R, N, K, t + 1 < iters ? &Q : nullptr);
+    out->refine_err.push_back(err);
+    if (t == 0 || err < *std::min_element(out->refine_err.begin(), out->refine_err.end() - 1)) {
+      out->L1p.swap(L1p);
+      out->L2.swap(L2);
+      out->R.swap(R);
     }
-    Q.swap(Y);                       // N x l, orthonormal columns
-    mul_at_q(Wh, N, K, Q, l, Z);     // Z = W_hat^T Q = B^T  (K x l)
-    // ---- Rayleigh-Ritz: eigen-decomposition of B B^T = Z^T Z (l x l)
-    std::vector<double> G(static_cast<size_t>(l) * l, 0.0);
-    for (int a = 0; a < l; ++a)
-      for (int b = a; b < l; ++b) {
-        double s = 0.0;
-        for (int k = 0; k < K; ++k) s += Z[static_cast<size_t>(k) * l + a] * Z[static_cast<size_t>(k) * l + b];
-        G[static_cast<size_t>(a) * l + b] = G[static_cast<size_t>(b) * l + a] = s;
-      }
-    std::vector<double> d, E;
-    jacobi_eigen(G, l, d, E);
-    // L2 = (Q E_r)^T, L1 = B^T E_r = Z E_r
-    for (int i = 0; i < r; ++i) {
-      for (int n = 0; n < N; ++n) {
-        double s = 0.0;
-        for (int a = 0; a < l; ++a) s += Q[static_cast<size_t>(n) * l + a] * E[static_cast<size_t>(a) * l + i];
-        L2d[static_cast<size_t>(i) * N + n] = s;
-      }
-      for (int k = 0; k < K; ++k) {
-        double s = 0.0;
-        for (int a = 0; a < l; ++a) s += Z[static_cast<size_t>(k) * l + a] * E[static_cast<size_t>(a) * l + i];
-        L1s[static_cast<size_t>(k) * r + i] = s;
-      }
-    }
-    // ---- 16-bit factors; the residual uses them as the runtime does
-    for (int k = 0; k < K; ++k)
-      for (int i = 0; i < r; ++i) {
-        const double v = static_cast<double>(out->inv_lam[k]) * L1s[static_cast<size_t>(k) * r + i];
-        const uint16_t b = f32_to_bf16_rne(static_cast<float>(v));
-        out->L1p[static_cast<size_t>(k) * r + i] = b;
-        L1s[static_cast<size_t>(k) * r + i] = static_cast<double>(bf16_to_f32(b)) / static_cast<double>(out->inv_lam[k]);
-      }
-    for (size_t i = 0; i < L2d.size(); ++i) {
-      const uint16_t b = f32_to_bf16_rne(static_cast<float>(L2d[i]));
-      out->L2[i] = b;
-      L2d[i] = bf16_to_f32(b);
-    }
+    if (t + 1 < iters)
+      parallel_for(N, [&](long b, long e) {
+        for (size_t i = static_cast<size_t>(b) * K; i < static_cast<size_t>(e) * K; ++i) A[i] = Wh[i] - Q[i];
+      });
   }
-  out->R.resize(static_cast<size_t>(N) * K);
-  parallel_for(N, [&](long b, long e) {
-    std::vector<double> l2n(std::max(r, 1));
-    for (long n = b; n < e; ++n) {
-      for (int i = 0; i < r; ++i) l2n[i] = L2d[static_cast<size_t>(i) * N + n];
-      for (int k = 0; k < K; ++k) {
-        double low = 0.0;
-        const double* l1 = &L1s[static_cast<size_t>(k) * r];
-        for (int i = 0; i < r; ++i) low += l1[i] * l2n[i];
-        out->R[static_cast<size_t>(n) * K + k] = static_cast<float>(Wh[static_cast<size_t>(n) * K + k] - low);
-      }
-    }
-  });
   return SVDQ_OK;
 }
 

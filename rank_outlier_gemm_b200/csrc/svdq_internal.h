@@ -90,6 +90,7 @@ struct HostSplit {
   std::vector<uint16_t> L1p;       // [K, r] bf16
   std::vector<uint16_t> L2;        // [r, N] bf16
   std::vector<float> R;            // [N, K]
+  std::vector<double> refine_err;  // ||R - Q(R)||_F of each split tried (refinement)
 };
 // Smoothing + randomized SVD split + residual on the host (float64 math).
 svdq_status host_prepare_split(const uint16_t* W_bf16, const float* act_absmax, int N, int K,
@@ -119,6 +120,7 @@ struct svdq_weights {
   std::vector<uint16_t> L2;      // [rank, N]
   std::vector<float> bias;
   std::vector<float> residual;   // [N, K] R / alpha_w (only if kept)
+  std::vector<double> refine_err;  // residual quantization error of each split tried by prepare
   // tensor maps over the weight-side buffers
   CUtensorMap map_l1{};
   CUtensorMap map_wq_256{}, map_wq_128{};

@@ -39,7 +39,7 @@ def test_host_only_helpers():
     assert B.svdq_act_sf_bytes(1, 3072) == 128 * 192
     assert B.svdq_act_sf_bytes(129, 64) == 256 * 4
     o = B.svdq_prepare_opts_default()
-    assert (o.alpha, o.rank, o.power_iters, o.oversample) == (0.5, 32, 4, 16)
+    assert (o.alpha, o.rank, o.power_iters, o.oversample, o.refine_iters) == (0.5, 32, 4, 16, 1)
     assert "sm_100a" in B.svdq_version()
 
 
@@ -57,6 +57,9 @@ def test_invalid_arguments_rejected_before_gpu():
     with pytest.raises(B.SvdqError) as e:   # rank above min(N, K)
         B.svdq_prepare_weights(W, np.ones(64, np.float32), rank=40)
     assert e.value.status == 1
+    with pytest.raises(B.SvdqError) as e:   # refinement needs at least one split
+        B.svdq_prepare_weights(W, np.ones(64, np.float32), rank=4, refine_iters=0)
+    assert e.value.status == 1 and "refine_iters" in str(e.value)
     bad = np.ones(64, np.float32)
     bad[3] = np.nan
     with pytest.raises(B.SvdqError) as e:

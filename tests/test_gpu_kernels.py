@@ -240,6 +240,33 @@ def test_library_prepare_invariants():
     assert e_lib < 1.5 * e_orc + 1e-3
 
 
+def test_library_refinement_matches_oracle():
+    """Refined split (SVDQuant §4.2, the survey's reading of its iterations):
+    the library's residual quantization errors follow the oracle's (exact SVD)
+    closely, the kept split is the one with the smallest error (recomputed by
+    the oracle from the exported residual), refinement lowers the error on the
+    outlier layer, and the refined layer meets the output tolerance."""
+    L = G.lib()
+    t, _ = _case_prep("tiny/layer", 64)
+    orc = OS.prepare(t.W, t.act_absmax, t.bias, 16, iters=4)
+    w = L.svdq_prepare_weights(t.W_bits, t.act_absmax, t.bias_bits, rank=16, keep_residual=True,
+                               refine_iters=4)
+    errs = L.svdq_weights_refine_errors(w)
+    assert len(errs) == 4
+    np.testing.assert_allclose(errs, orc.refine_errors, rtol=2e-2)
+    assert min(errs) < 0.95 * errs[0]
+    ex = L.svdq_weights_export(w, residual=True)
+    R = (ex["residual"].astype(np.float64) * ex["alpha_w"]).astype(np.float32)
+    kept = np.linalg.norm(R.astype(np.float64) - OS.fake_quantize_weights(R))
+    assert kept == pytest.approx(min(errs), rel=1e-9)
+    plain = L.svdq_prepare_weights(t.W_bits, t.act_absmax, t.bias_bits, rank=16)
+    assert len(L.svdq_weights_refine_errors(plain)) == 1
+    prep = OS.prepare_from_factors(OS.smooth_weight(t.W, ex["inv_lam"]), ex["inv_lam"],
+                                   OF.bf16_bits_to_f64(ex["L1p"]), OF.bf16_bits_to_f64(ex["L2"]), t.bias)
+    Y, _ = G.run_layer(w, t.X_bits)
+    G.check_Y(Y, OS.linear(prep, t.X))
+
+
 def test_bounded_wait_reports_timeout():
     L = G.lib()
     t, prep = _case_prep("tiny/layer", 64)

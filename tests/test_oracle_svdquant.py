@@ -186,3 +186,51 @@ def test_lora_concat_equals_separate_sum_and_keeps_codes():
     assert both.alpha_w == prep.alpha_w and both.rank == 48
     sep = S.linear(prep, t.X) + 0.75 * (t.X.astype(np.float64) @ A) @ B
     assert _rel(S.linear(both, t.X), sep) < 1e-12
+
+
+def _tiny_case():
+    case = config_cases("tiny")[0]
+    return case, make_layer_inputs(case)
+
+
+def test_refinement_keeps_the_best_split_and_one_iteration_is_plain():
+    """Step 4b (SVDQuant §4.2, refinement over several iterations): iters = 1 is
+    the plain split; with more iterations the kept split is the one with the
+    smallest residual quantization error, its first error is the plain split's,
+    and the kept split still reconstructs W_hat exactly before quantization."""
+    case, t = _tiny_case()
+    plain = S.prepare(t.W, t.act_absmax, t.bias, case.rank)
+    assert len(plain.refine_errors) == 1
+    ref = S.prepare(t.W, t.act_absmax, t.bias, case.rank, iters=4)
+    errs = ref.refine_errors
+    assert len(errs) == 4
+    assert errs[0] == pytest.approx(plain.refine_errors[0], rel=0, abs=0)
+    q = S.fake_quantize_weights(ref.R)
+    assert np.linalg.norm(ref.R.astype(np.float64) - q) == pytest.approx(min(errs), rel=1e-12)
+    # the outlier layer gains from refinement (the qualitative claim of §4.2)
+    assert min(errs) < 0.95 * errs[0]
+    W_hat = S.smooth_weight(t.W, ref.inv_lam)
+    low = (ref.L1p / ref.inv_lam.astype(np.float64)[:, None]) @ ref.L2b
+    np.testing.assert_allclose(low.T + ref.R.astype(np.float64), W_hat, rtol=0, atol=1e-6)
+
+
+def test_refinement_of_an_exactly_low_rank_weight_stays_put():
+    """A smoothed weight of rank r is split exactly by the SVD: every iterate's
+    residual is only the 16-bit rounding of the factors, so all errors are tiny
+    compared with quantizing the weight itself."""
+    rng = np.random.default_rng(3)
+    N, K, r = 96, 128, 8
+    W = (rng.normal(0, 1, (N, r)) @ rng.normal(0, 0.05, (r, K))).astype(np.float32)
+    absmax = np.ones(K, np.float32)
+    prep = S.prepare(W, absmax, None, r, iters=3)
+    W_hat = S.smooth_weight(W, prep.inv_lam)
+    full = np.linalg.norm(W_hat - S.fake_quantize_weights(W_hat.astype(np.float32)))
+    assert max(prep.refine_errors) < 1e-2 * full
+
+
+def test_fake_quantize_weights_is_the_codec_round_trip():
+    """Q(R) = alpha_w * dequantize(quantize(R / alpha_w)) (App. A.2: Q(R) = s_R Q_R);
+    on a residual already on the FP4 grid times a power of two it is exact."""
+    _, _, _, W = make_fp4_grid_inputs(16, 64, 32, seed=5)
+    R = (W * np.float32(2.0 ** -9)).astype(np.float32)
+    np.testing.assert_array_equal(S.fake_quantize_weights(R), R.astype(np.float64))
