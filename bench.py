@@ -248,6 +248,20 @@ def refinement(L, iters=4):
     return out
 
 
+def alpha_search(L, rows=256):
+    """NEXT-3 (App. D migration strength): relative output error per candidate
+    alpha on a calibration batch of one FLUX layer, through the library's own
+    preparation and kernels, and the search's wall time."""
+    c = [x for x in config_cases("flux") if x.name == "attn_out"][0]
+    t = make_layer_inputs(c)
+    alphas = (0.3, 0.4, 0.5, 0.6, 0.7, 0.8, 0.9)
+    t0 = time.time()
+    errs, best = L.svdq_search_alpha(t.W_bits, t.X_bits[:rows], t.bias_bits, alphas, rank=c.rank)
+    return {"layer": f"{c.label} N={c.N} K={c.K} rank={c.rank}, calibration rows {rows}",
+            "rel_err": dict(zip([str(a) for a in alphas], errs)), "best_alpha": alphas[best],
+            "gain_vs_0.5": 1.0 - errs[best] / errs[alphas.index(0.5)], "search_s": time.time() - t0}
+
+
 # ------------------------------------------------------------------ ours
 def run_ours(args):
     import torch
@@ -339,7 +353,7 @@ def run_ours(args):
 
     # low-rank overhead: the same kernels at rank 0 (extras)
     overhead = None
-    unfused = sweep = small = refine = None
+    unfused = sweep = small = refine = asearch = None
     if args.extras:
         def step0():
             for l in layers:
@@ -363,6 +377,7 @@ def run_ours(args):
             sweep = rank_sweep(L, torch, layers, dev, stream)
             small = small_m(L, torch, dev, stream)
             refine = refinement(L)
+            asearch = alpha_search(L)
 
     # end to end through the public host-buffer call: H2D of X, both kernels, D2H of Y
     e2e = None
@@ -415,6 +430,7 @@ def run_ours(args):
             "rank_sweep": sweep,
             "small_m_lora": small,
             "refinement": refine,
+            "alpha_search": asearch,
             "gpu_launches": 2 * nl * args.steps,
             "e2e": e2e,
         }

@@ -101,6 +101,25 @@ svdq_status svdq_prepare_weights(const uint16_t* W_bf16, const float* act_absmax
                                  svdq_weights** out);
 
 /*
+ * Per-layer choice of the smoothing strength (App. D: alpha sets how much of
+ * the activation range migrates into the weights; 0.5 by default).  For each
+ * of the n_alpha candidates in `alphas` (each in [0, 1]) the layer is prepared
+ * as svdq_prepare_weights does with opts->alpha = alphas[i] and the per-channel
+ * maxima of the calibration batch, both kernels run on the batch, and
+ * rel_err[i] = ||Y_i - (X W^T + b)||_F / ||X W^T + b||_F with the reference
+ * accumulated in fp32 on the device.  *best is the index of the smallest
+ * error.  Synchronous; allocates and frees its own device buffers.
+ *   W_bf16     host, N x K bf16
+ *   X_bf16     host, M x K bf16 calibration activations
+ *   bias_bf16  host, N bf16, or NULL
+ *   opts       NULL for the defaults (its alpha is ignored)
+ *   rel_err    host, n_alpha doubles (out);  best  host int (out)
+ */
+svdq_status svdq_search_alpha(const uint16_t* W_bf16, const uint16_t* X_bf16, int M, const uint16_t* bias_bf16,
+                              int N, int K, const float* alphas, int n_alpha, const svdq_prepare_opts* opts,
+                              void* stream, double* rel_err, int* best);
+
+/*
  * The residual quantization error ||R - Q(R)||_F (Frobenius, float64, in the
  * smoothed-weight space) of each split svdq_prepare_weights tried, in order:
  * one value without refinement, refine_iters values with it (the kept split

@@ -165,6 +165,24 @@ def prepare(W, act_absmax, bias, rank: int, alpha: float = 0.5, iters: int = 1) 
     return best
 
 
+def search_alpha(W, X, bias, rank: int, alphas, iters: int = 1):
+    """Per-layer smoothing strength (App. D: alpha is the migration strength of
+    the smoothing; the survey's NEXT-3 reading): for each candidate, prepare
+    with the calibration batch's per-channel maxima and score the layer output
+    by ||Y - (X W^T + b)||_F / ||X W^T + b||_F in float64.  Returns (errors,
+    index of the smallest)."""
+    X = np.asarray(X, np.float32)
+    exact = X.astype(np.float64) @ np.asarray(W, np.float64).T
+    if bias is not None:
+        exact = exact + np.asarray(bias, np.float64)[None, :]
+    absmax = np.abs(X).max(axis=0)
+    errs = []
+    for a in alphas:
+        prep = prepare(W, absmax, bias, rank, alpha=float(a), iters=iters)
+        errs.append(float(np.linalg.norm(linear(prep, X) - exact) / np.linalg.norm(exact)))
+    return errs, int(np.argmin(errs))
+
+
 def smooth_activations(X, inv_lam) -> np.ndarray:
     """X_hat = fp32(x * inv_lam) elementwise (one fp32 rounding)."""
     return (np.asarray(X, np.float32) * np.asarray(inv_lam, np.float32)[None, :]).astype(np.float32)

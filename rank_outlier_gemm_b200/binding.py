@@ -60,6 +60,8 @@ _SIGS = {
     "svdq_check_device_errors": (_i, [_vp]),
     "svdq_selftest_codec": (_i, [ctypes.POINTER(ctypes.c_uint)]),
     "svdq_weights_refine_errors": (_i, [_vp, ctypes.POINTER(ctypes.c_double), _i, ctypes.POINTER(_i)]),
+    "svdq_search_alpha": (_i, [_vp, _vp, _i, _vp, _i, _i, _vp, _i, ctypes.POINTER(PrepareOpts), _vp,
+                               ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i)]),
     "svdq_debug_launch_stalled_act": (_i, [_vp, _vp, _i, _vp, _vp, _vp, _vp]),
     "svdq_last_error": (ctypes.c_char_p, []),
     "svdq_version": (ctypes.c_char_p, []),
@@ -262,6 +264,23 @@ def svdq_weights_export(w: Weights, residual: bool = False) -> dict:
 
 def svdq_set_wait_limit_ns(ns: int) -> None:
     _lib.svdq_set_wait_limit_ns(int(ns))
+
+
+def svdq_search_alpha(W_bf16, X_bf16, bias_bf16=None, alphas=(0.3, 0.4, 0.5, 0.6, 0.7, 0.8), rank: int = 32,
+                      refine_iters: int = 1, stream=None):
+    """(relative output error per alpha, index of the best) on the calibration batch X."""
+    Wp, Wk = _host(W_bf16, np.uint16)
+    Xp, Xk = _host(X_bf16, np.uint16)
+    bp, bk = _host(bias_bf16, np.uint16)
+    N, K = Wk.shape
+    a = np.ascontiguousarray(np.asarray(alphas, np.float32))
+    o = svdq_prepare_opts_default()
+    o.rank, o.refine_iters = rank, refine_iters
+    err = (ctypes.c_double * len(a))()
+    best = ctypes.c_int(0)
+    _check(_lib.svdq_search_alpha(Wp, Xp, Xk.shape[0], bp, N, K, a.ctypes.data, len(a), ctypes.byref(o),
+                                  _stream(stream), err, ctypes.byref(best)), "svdq_search_alpha")
+    return [float(err[i]) for i in range(len(a))], int(best.value)
 
 
 def svdq_weights_refine_errors(w: Weights) -> list:

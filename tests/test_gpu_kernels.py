@@ -267,6 +267,22 @@ def test_library_refinement_matches_oracle():
     G.check_Y(Y, OS.linear(prep, t.X))
 
 
+def test_library_alpha_search_matches_oracle():
+    """NEXT-3 alpha search (App. D migration strength) run through the library's
+    preparation and kernels: the per-candidate output errors follow the
+    oracle's float64 ones, and the chosen alpha's error is the oracle's minimum
+    up to the spread of near-ties."""
+    L = G.lib()
+    t, _ = _case_prep("tiny/layer", 64)
+    alphas = [0.0, 0.25, 0.5, 0.75, 0.9]
+    errs, best = L.svdq_search_alpha(t.W_bits, t.X_bits, t.bias_bits, alphas, rank=16)
+    ref, ref_best = OS.search_alpha(t.W, t.X, t.bias, 16, alphas)
+    np.testing.assert_allclose(errs, ref, rtol=3e-2)
+    assert best == int(np.argmin(errs))
+    assert errs[best] <= 1.02 * min(ref)
+    assert errs[2] < errs[0]
+
+
 def test_bounded_wait_reports_timeout():
     L = G.lib()
     t, prep = _case_prep("tiny/layer", 64)

@@ -234,3 +234,20 @@ def test_fake_quantize_weights_is_the_codec_round_trip():
     _, _, _, W = make_fp4_grid_inputs(16, 64, 32, seed=5)
     R = (W * np.float32(2.0 ** -9)).astype(np.float32)
     np.testing.assert_array_equal(S.fake_quantize_weights(R), R.astype(np.float64))
+
+
+def test_alpha_search_scores_each_candidate_and_picks_the_smallest():
+    """NEXT-3 (App. D migration strength): each candidate's error is the plain
+    prepare-then-linear error at that alpha, the pick is the smallest, and on
+    the outlier layer migrating some activation range into the weights beats
+    none (alpha = 0 leaves the x40 outlier channels in the activations)."""
+    case, t = _tiny_case()
+    X = t.X[:32]
+    alphas = [0.0, 0.5, 0.8]
+    errs, best = S.search_alpha(t.W, X, t.bias, case.rank, alphas)
+    exact = X.astype(np.float64) @ t.W.astype(np.float64).T + t.bias
+    p5 = S.prepare(t.W, np.abs(X).max(axis=0), t.bias, case.rank, alpha=0.5)
+    e5 = np.linalg.norm(S.linear(p5, X) - exact) / np.linalg.norm(exact)
+    assert errs[1] == pytest.approx(e5, rel=1e-12)
+    assert best == int(np.argmin(errs))
+    assert errs[1] < 0.5 * errs[0]
