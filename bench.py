@@ -137,6 +137,31 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(sm)}
 
 
+# ------------------------------------------------------------------ ranks
+def dist_env():
+    """(world size, rank, local rank) as a torchrun launch sets them; 1, 0, 0 alone."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest x over all ranks (each rank's own device time of the same
+    timed region; the slowest rank sets the job's time)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(flops_per_rank_step: float, ms_step: float, world: int) -> float:
+    """Whole-job TFLOP/s of independent replicas: every rank's work over the
+    slowest rank's step time (weak scaling)."""
+    return world * flops_per_rank_step / (ms_step * 1e-3) / 1e12
+
+
 # ------------------------------------------------------------------ extras
 def _time_ms(torch, stream, fn, reps):
     for _ in range(3):
@@ -267,9 +292,7 @@ def run_ours(args):
     import torch
     import torch.distributed as dist
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = dist_env()
     torch.cuda.set_device(local)
     if world > 1:
         dist.init_process_group("nccl", device_id=torch.device("cuda", local))
@@ -305,12 +328,8 @@ def run_ours(args):
             dist.barrier()
         torch.cuda.synchronize()
 
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def slowest(x: float) -> float:
+        return max_over_ranks(x, world, dev)
 
     for _ in range(args.warmup):
         step()
@@ -327,12 +346,12 @@ def run_ours(args):
         t1.record(stream)
         barrier()
     assert L.svdq_check_device_errors() == 0
-    ms = max_over_ranks(t0.elapsed_time(t1))
+    ms = slowest(t0.elapsed_time(t1))
     ms_step = ms / args.steps
     k1 = [statistics.mean(evs[s][i][0].elapsed_time(evs[s][i][1]) for s in range(args.steps)) for i in range(nl)]
     k2 = [statistics.mean(evs[s][i][1].elapsed_time(evs[s][i][2]) for s in range(args.steps)) for i in range(nl)]
     flops_step = sum(l["case"].flops for l in layers)
-    value = world * flops_step / (ms_step * 1e-3) / 1e12
+    value = job_throughput(flops_step, ms_step, world)
 
     pk = peaks()
     # The burst cuBLAS figure applies while the SM clock holds its maximum; a run that
@@ -402,10 +421,10 @@ def run_ours(args):
             step_e2e()
         b.record(stream)
         barrier()
-        ems = max_over_ranks(a.elapsed_time(b)) / args.e2e_steps
+        ems = slowest(a.elapsed_time(b)) / args.e2e_steps
         h2d = sum(l["case"].M * l["case"].K * 2 for l in layers)
         d2h = sum(l["case"].M * l["case"].N * 2 for l in layers)
-        e2e = {"value": world * flops_step / (ems * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ems,
+        e2e = {"value": job_throughput(flops_step, ems, world), "unit": "TFLOP/s", "ms_per_step": ems,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
 
     if rank == 0:
@@ -484,9 +503,8 @@ def run_reference(args):
     """The oracle as the reference arm: each step computes a bounded sample of
     the step's outputs (args.ref_rows rows x args.ref_cols output columns of
     every layer) on the host cores; flops count only the sampled outputs."""
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    if rank != 0:
+    world, rank, _ = dist_env()
+    if rank != 0:  # the host-side reference runs once per job, on rank 0
         return
     from oracle import svdquant as OS
     preps = _oracle_layers()
