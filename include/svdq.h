@@ -26,6 +26,10 @@
  *    buffers alive until the work queued on the stream has finished.  The
  *    library owns the svdq_weights handle and the device memory inside it;
  *    svdq_weights_destroy frees both.
+ *  - CUDA graphs: the runtime calls (both kernels, svdq_forward and its
+ *    allocation-free variant) can be captured into a graph once the same call
+ *    has run eagerly on the device, since a first call sets up per-device
+ *    state (error word, kernel attributes, occupancy queries).
  *  - Streams: `stream` is a cudaStream_t passed as void* (NULL = the legacy
  *    default stream).  Runtime calls only enqueue work; they do not
  *    synchronize.  Weight preparation and LoRA attachment synchronize.
@@ -185,6 +189,13 @@ svdq_status svdq_quantize_act_lowrank_down(const svdq_weights* w, const void* X_
  * accumulated in fp32 in tensor memory.
  *   xq, xsf, T  as written by svdq_quantize_act_lowrank_down for the same M
  *   Y_bf16      device, M x N bf16
+ * When the 128 x 256 output tiles would leave most SMs idle (small M), K is
+ * split over a cluster of up to 8 CTAs per tile and the fp32 partials are
+ * summed in a fixed order through distributed shared memory; the result is
+ * then deterministic but its rounding differs from the unsplit sum within
+ * fp32 accumulation error.  The launch is a programmatic dependent of the
+ * kernel ahead of it in the stream: it reads xq, xsf and T only once that
+ * kernel has completed.
  */
 svdq_status svdq_linear_w4a4(const svdq_weights* w, const void* xq, const void* xsf,
                              const void* T, int M, void* Y_bf16, void* stream);
@@ -287,6 +298,16 @@ svdq_status svdq_check_device_errors(void* stream);
  */
 svdq_status svdq_debug_launch_stalled_act(const svdq_weights* w, const void* X_bf16, int M,
                                           void* xq, void* xsf, void* T, void* stream);
+
+/*
+ * Test hook: svdq_linear_w4a4 with the split-K factor fixed to `ksplit` CTAs
+ * per output tile (1 = no split) instead of the automatic choice.  The split
+ * is clamped to the number of 256-wide K tiles; a split whose clusters would
+ * not all be resident at once falls back to 1.  SVDQ_ERR_INVALID_ARG unless
+ * 1 <= ksplit <= 8; otherwise as svdq_linear_w4a4.
+ */
+svdq_status svdq_debug_linear_w4a4_ksplit(const svdq_weights* w, const void* xq, const void* xsf,
+                                          const void* T, int M, void* Y_bf16, int ksplit, void* stream);
 
 /*
  * Device self-test of the NVFP4 group encoder's exact shortcuts (both kernels

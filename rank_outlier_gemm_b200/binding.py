@@ -63,6 +63,7 @@ _SIGS = {
     "svdq_search_alpha": (_i, [_vp, _vp, _i, _vp, _i, _i, _vp, _i, ctypes.POINTER(PrepareOpts), _vp,
                                ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i)]),
     "svdq_debug_launch_stalled_act": (_i, [_vp, _vp, _i, _vp, _vp, _vp, _vp]),
+    "svdq_debug_linear_w4a4_ksplit": (_i, [_vp, _vp, _vp, _vp, _i, _vp, _i, _vp]),
     "svdq_last_error": (ctypes.c_char_p, []),
     "svdq_version": (ctypes.c_char_p, []),
 }
@@ -200,6 +201,13 @@ def svdq_debug_launch_stalled_act(w: Weights, X, xq, xsf, T, stream=None) -> Non
 def svdq_linear_w4a4(w: Weights, xq, xsf, T, M: int, Y: torch.Tensor, stream=None) -> None:
     _check(_lib.svdq_linear_w4a4(w.handle, _dev(xq, "xq"), _dev(xsf, "xsf"), _dev(T, "T"), M, _dev(Y, "Y"),
                                  _stream(stream)), "svdq_linear_w4a4")
+
+
+def svdq_debug_linear_w4a4_ksplit(w: Weights, xq, xsf, T, M: int, Y: torch.Tensor, ksplit: int,
+                                  stream=None) -> None:
+    _check(_lib.svdq_debug_linear_w4a4_ksplit(w.handle, _dev(xq, "xq"), _dev(xsf, "xsf"), _dev(T, "T"), M,
+                                              _dev(Y, "Y"), ksplit, _stream(stream)),
+           "svdq_debug_linear_w4a4_ksplit")
 
 
 def svdq_forward(w: Weights, X: torch.Tensor, Y: torch.Tensor, workspace: torch.Tensor, stream=None) -> None:

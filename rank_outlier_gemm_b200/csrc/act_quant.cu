@@ -93,6 +93,9 @@ __global__ void __launch_bounds__(kThreads, 2) act_quant_lowrank_kernel(
   const int nt = base + (split < rem ? 1 : 0);
   const int t0 = split * base + min(split, rem);
   const bool lowrank = p.r_pad > 0;
+  // the GEMM behind this kernel may start its set-up and weight loads now; it
+  // waits for this grid to finish before reading what this kernel writes
+  grid_dep_launch_dependents();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {

@@ -420,6 +420,19 @@ svdq_status svdq_linear_w4a4(const svdq_weights* w, const void* xq, const void* 
   return launch_gemm_w4a4(a, static_cast<cudaStream_t>(stream));
 }
 
+svdq_status svdq_debug_linear_w4a4_ksplit(const svdq_weights* w, const void* xq, const void* xsf, const void* T,
+                                          int M, void* Y_bf16, int ksplit, void* stream) {
+  if (ksplit < 1 || ksplit > 8) return fail(SVDQ_ERR_INVALID_ARG, "ksplit=%d must be in [1, 8]", ksplit);
+  SVDQ_TRY(check_runtime(w, M));
+  SVDQ_TRY(check_dev_ptr(xq, "xq"));
+  SVDQ_TRY(check_dev_ptr(xsf, "xsf"));
+  SVDQ_TRY(check_dev_ptr(Y_bf16, "Y"));
+  if (w->r_pad > 0) SVDQ_TRY(check_dev_ptr(T, "T"));
+  GemmArgs a{M, w->N, w->K, w->r_pad, xq, xsf, T, &w->map_wq_256, &w->map_wq_128, &w->map_l2_256,
+             &w->map_l2_128, w->d_wsf, w->d_bias, w->alpha_w, Y_bf16, ksplit};
+  return launch_gemm_w4a4(a, static_cast<cudaStream_t>(stream));
+}
+
 size_t svdq_act_codes_bytes(int M, int K) {
   return M > 0 && K > 0 ? static_cast<size_t>(M) * K / 2 : 0;
 }

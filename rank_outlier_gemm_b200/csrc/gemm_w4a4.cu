@@ -23,6 +23,18 @@
 // of acc[(j+1)%2], which the epilogue of tile j-1 releases first; so the
 // epilogue of one tile runs under the main loop of the next, and the slab MMAs,
 // which need no scales, keep the tensor pipe busy during that hand-over.
+//
+// Few output tiles (small M): split-K.  A cluster of S CTAs shares one tile,
+// each CTA accumulating a contiguous range of K tiles (the last split also
+// takes the low-rank slab); the partial accumulators go to shared memory and,
+// after a cluster barrier, each CTA sums a slice of the tile's rows over the S
+// partials through distributed shared memory in split order (0, 1, ..., S-1),
+// so the result does not depend on timing.
+//
+// The kernel is launched as a programmatic dependent of the kernel ahead of
+// it in the stream (the activation kernel): its set-up and the weight-side
+// loads of the first stages run before that kernel has finished, and the
+// producer waits for it only before loading activation codes, scales and T.
 #include <algorithm>
 #include <cstddef>
 
@@ -44,6 +56,9 @@ constexpr int kSfb = 2 * 2048;                  // two 128-row blocks x four ato
 constexpr int kStage = kATile + kBTile + kSfa + kSfb;
 constexpr int kSfCols = 16 + 32;                // TMEM columns of one scale slot (one K tile)
 constexpr int kSfSlots = 2;                     // 2 x 48 = 96 columns
+constexpr int kMaxSplit = 8;                    // portable cluster size
+constexpr int kPartStride = kBN + 4;            // fp32 words per partial row (bank spread)
+static_assert(128 * kPartStride * 4 <= kStages * kStage, "partials fit in the stage buffers");
 
 struct K2Params {
   int M, N, K, r_pad;
@@ -52,6 +67,7 @@ struct K2Params {
   int nblk_total;  // ceil(N / 128)
   int slab;        // ceil(r_pad / 32)
   int mtiles, ntiles;
+  int ksplit;      // CTAs (one cluster) per output tile along K; 1 = persistent
   const uint8_t* xsf;
   const uint8_t* wsf;
   const float* bias;
@@ -117,6 +133,45 @@ __device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], const float
   }
 }
 
+// Split-K: this CTA's share of the tile's rows, summed over the S partials in
+// split order, then y = alpha_w * acc + b in bf16 RNE.
+__device__ __forceinline__ void split_reduce(const K2Params& p, const float* part, int split, int t) {
+  const int m0 = (t % p.mtiles) * 128, n0 = (t / p.mtiles) * kBN;
+  const int rows = min(128, p.M - m0);
+  const int per = (rows + p.ksplit - 1) / p.ksplit;
+  const int r_lo = split * per, r_hi = min(rows, r_lo + per);
+  const uint32_t base = smem_u32(part);
+  for (int i = threadIdx.x; i < (r_hi - r_lo) * (kBN / 4); i += kThreads) {
+    const int r = r_lo + i / (kBN / 4), c = 4 * (i % (kBN / 4));
+    const int n = n0 + c;
+    if (n >= p.N) continue;
+    const uint32_t off = static_cast<uint32_t>(r * kPartStride + c) * 4u;
+    float4 v[kMaxSplit];
+#pragma unroll
+    for (int q = 0; q < kMaxSplit; ++q)
+      if (q < p.ksplit) v[q] = ld_dsmem_f4(mapa_shared(base + off, q));
+    float4 acc = v[0];
+#pragma unroll
+    for (int q = 1; q < kMaxSplit; ++q)
+      if (q < p.ksplit) {
+        acc.x = __fadd_rn(acc.x, v[q].x);
+        acc.y = __fadd_rn(acc.y, v[q].y);
+        acc.z = __fadd_rn(acc.z, v[q].z);
+        acc.w = __fadd_rn(acc.w, v[q].w);
+      }
+    const float4 b = *reinterpret_cast<const float4*>(p.bias + n);
+    const float y0 = __fadd_rn(__fmul_rn(acc.x, p.alpha_w), b.x);
+    const float y1 = __fadd_rn(__fmul_rn(acc.y, p.alpha_w), b.y);
+    const float y2 = __fadd_rn(__fmul_rn(acc.z, p.alpha_w), b.z);
+    const float y3 = __fadd_rn(__fmul_rn(acc.w, p.alpha_w), b.w);
+    const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(y0)) |
+                        (uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(y1))) << 16);
+    const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(y2)) |
+                        (uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(y3))) << 16);
+    *reinterpret_cast<uint2*>(p.Y + static_cast<size_t>(m0 + r) * p.N + n) = make_uint2(lo, hi);
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
     const __grid_constant__ CUtensorMap map_xq, const __grid_constant__ CUtensorMap map_wq,
     const __grid_constant__ CUtensorMap map_t, const __grid_constant__ CUtensorMap map_l2,
@@ -129,7 +184,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
 
   const uint32_t warp = warp_id(), lane = lane_id();
   const int ntiles_total = p.mtiles * p.ntiles;
-  const int per_tile = p.kt + p.slab;
+  // split-K: CTA blockIdx.x is rank (blockIdx.x % S) of the cluster that owns
+  // tile blockIdx.x / S; it takes a contiguous range of the K tiles, and the
+  // last split the slab as well (its range is never the longer one)
+  const int S = p.ksplit;
+  const int split = static_cast<int>(blockIdx.x) % S;
+  const int tile0 = static_cast<int>(blockIdx.x) / S, tile_step = static_cast<int>(gridDim.x) / S;
+  const int kt_base = p.kt / S, kt_rem = p.kt % S;
+  const int kt_lo = split * kt_base + min(split, kt_rem);
+  const int nslab = split == S - 1 ? p.slab : 0;
+  const int per_tile = nslab + kt_base + (split < kt_rem ? 1 : 0);
+  float* part = reinterpret_cast<float*>(smem);  // split-K partials, after the tile's MMAs
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -168,39 +233,63 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
         tma_prefetch_desc(&map_t);
         tma_prefetch_desc(&map_l2);
       }
+      // A stage's loads come in two halves: the weight side (codes, scales,
+      // L2), which no kernel of the forward pass writes, and the activation
+      // side (codes, scales, T) from the kernel ahead.  The first stages'
+      // weight halves go out before the wait for that kernel.
+      int m0 = (tile0 % p.mtiles) * 128, n0 = (tile0 / p.mtiles) * kBN;
+      int nb_valid = min(2, p.nblk_total - n0 / 128);
+      const int npre = tile0 < ntiles_total ? min(kStages, per_tile) : 0;
+      for (int k = 0; k < npre; ++k) {
+        uint8_t* st = smem + k * kStage;
+        if (k >= nslab) {
+          const int kk = kt_lo + k - nslab;
+          const int nkb = min(4, p.kb_total - 4 * kk);
+          mbar_arrive_expect_tx(&sh->full[k], kATile + kBTile + 512u * nkb * (1 + nb_valid));
+          tma_load_2d(st + kATile, &map_wq, &sh->full[k], kk * 128, n0);
+          for (int nb = 0; nb < nb_valid; ++nb)
+            bulk_load(st + kATile + kBTile + kSfa + nb * 2048,
+                      p.wsf + (static_cast<size_t>(n0 / 128 + nb) * p.kb_total + 4 * kk) * 512, 512u * nkb,
+                      &sh->full[k]);
+        } else {
+          mbar_arrive_expect_tx(&sh->full[k], kATile + kBN * 64);
+          tma_load_2d(st + kATile, &map_l2, &sh->full[k], 32 * k, n0);
+        }
+      }
+      grid_dep_wait();
       int it = 0;
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < ntiles_total; t += gridDim.x) {
-        const int m0 = (t % p.mtiles) * 128;
-        const int n0 = (t / p.mtiles) * kBN;
-        int nb_valid = 0;
-        for (int nb = 0; nb < 2; ++nb) nb_valid += (n0 / 128 + nb < p.nblk_total);
+      for (int t = tile0; ok && t < ntiles_total; t += tile_step) {
+        m0 = (t % p.mtiles) * 128;
+        n0 = (t / p.mtiles) * kBN;
+        nb_valid = min(2, p.nblk_total - n0 / 128);
         for (int k = 0; k < per_tile; ++k, ++it) {
           const int s = it % kStages;
           const uint32_t ph = (it / kStages) & 1;
-          if (!wait_bounded(&sh->empty[s], ph ^ 1, wc)) {
+          const bool pre = it < npre;  // weight half already issued
+          if (!pre && !wait_bounded(&sh->empty[s], ph ^ 1, wc)) {
             ok = false;
             break;
           }
           uint8_t* st = smem + s * kStage;
-          if (k >= p.slab) {
-            const int kk = k - p.slab;
+          if (k >= nslab) {
+            const int kk = kt_lo + k - nslab;
             const int nkb = min(4, p.kb_total - 4 * kk);
-            mbar_arrive_expect_tx(&sh->full[s], kATile + kBTile + 512u * nkb * (1 + nb_valid));
+            if (!pre) mbar_arrive_expect_tx(&sh->full[s], kATile + kBTile + 512u * nkb * (1 + nb_valid));
             tma_load_2d(st, &map_xq, &sh->full[s], kk * 128, m0);
-            tma_load_2d(st + kATile, &map_wq, &sh->full[s], kk * 128, n0);
+            if (!pre) tma_load_2d(st + kATile, &map_wq, &sh->full[s], kk * 128, n0);
             bulk_load(st + kATile + kBTile,
                       p.xsf + (static_cast<size_t>(m0 / 128) * p.kb_total + 4 * kk) * 512, 512u * nkb,
                       &sh->full[s]);
-            for (int nb = 0; nb < nb_valid; ++nb)
-              bulk_load(st + kATile + kBTile + kSfa + nb * 2048,
-                        p.wsf + (static_cast<size_t>(n0 / 128 + nb) * p.kb_total + 4 * kk) * 512,
-                        512u * nkb, &sh->full[s]);
+            if (!pre)
+              for (int nb = 0; nb < nb_valid; ++nb)
+                bulk_load(st + kATile + kBTile + kSfa + nb * 2048,
+                          p.wsf + (static_cast<size_t>(n0 / 128 + nb) * p.kb_total + 4 * kk) * 512,
+                          512u * nkb, &sh->full[s]);
           } else {
-            const int j = k;
-            mbar_arrive_expect_tx(&sh->full[s], kATile + kBN * 64);
-            tma_load_2d(st, &map_t, &sh->full[s], 64 * j, m0);
-            tma_load_2d(st + kATile, &map_l2, &sh->full[s], 32 * j, n0);
+            if (!pre) mbar_arrive_expect_tx(&sh->full[s], kATile + kBN * 64);
+            tma_load_2d(st, &map_t, &sh->full[s], 64 * k, m0);
+            if (!pre) tma_load_2d(st + kATile, &map_l2, &sh->full[s], 32 * k, n0);
           }
         }
       }
@@ -222,7 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
       const uint64_t dl0 = desc_kmajor_sw64(stage0 + kATile);
       int it = 0, sfi = 0, j = 0;
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < ntiles_total; t += gridDim.x, ++j) {
+      for (int t = tile0; ok && t < ntiles_total; t += tile_step, ++j) {
         const int a = j & 1;
         if (!wait_bounded(&sh->acc_empty[a], ((j >> 1) & 1) ^ 1, wc)) break;
         tc_fence_after();
@@ -233,8 +322,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
           const int s = it % kStages;
           const uint32_t ph = (it / kStages) & 1;
           const uint64_t soff = static_cast<uint64_t>(s * (kStage >> 4));
-          if (k >= p.slab) {
-            const int nkb = min(4, p.kb_total - 4 * (k - p.slab));
+          if (k >= nslab) {
+            const int nkb = min(4, p.kb_total - 4 * (kt_lo + k - nslab));
             const int b = sfi & (kSfSlots - 1);
             // the writers waited for this stage's data before publishing its scales
             if (!wait_bounded(&sh->sf_full[b], (sfi / kSfSlots) & 1, wc)) {
@@ -282,13 +371,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     int it = 0, sfi = 0, j = 0;
     bool ok = true;
-    for (int t = blockIdx.x; ok && t < ntiles_total; t += gridDim.x, ++j) {
+    for (int t = tile0; ok && t < ntiles_total; t += tile_step, ++j) {
       const int a = j & 1;
       const uint32_t sf_region = tmem + (a ^ 1) * 256 + lane_off;
       for (int k = 0; k < per_tile; ++k, ++it) {
         const int s = it % kStages;
         const uint32_t ph = (it / kStages) & 1;
-        if (k == p.slab) {
+        if (k == nslab) {
           // the scale buffers live in acc[a^1]: wait until the previous tile's
           // epilogue has read its first 96 columns
           if (!wait_warp(&sh->sfreg_free[a ^ 1], ((j - 1) >> 1) & 1, wc)) {
@@ -296,7 +385,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
             break;
           }
         }
-        if (k >= p.slab) {
+        if (k >= nslab) {
           if (!wait_warp(&sh->full[s], ph, wc)) {
             ok = false;
             break;
@@ -353,7 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     const int row = q * 32 + lane;
     int j = 0;
-    for (int t = blockIdx.x; t < ntiles_total; t += gridDim.x, ++j) {
+    for (int t = tile0; t < ntiles_total; t += tile_step, ++j) {
       const int a = j & 1;
       const int m = (t % p.mtiles) * 128 + row;
       const int n0 = (t / p.mtiles) * kBN;
@@ -368,6 +457,30 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
       __syncwarp();
       if (!wait_warp(&sh->acc_full[a], (j >> 1) & 1, wc)) break;
       tc_fence_after();
+      if (S > 1) {
+        // split-K (one tile per CTA): this split's partial rows into the
+        // stage buffers, which the tile's completed MMAs no longer read
+        float* prow = part + row * kPartStride;
+        for (int c = 0; c < kBN / 32; ++c) {
+          uint32_t rr[32];
+          tmem_ld_x32(tmem + a * 256 + lane_off + 32 * c, rr);
+          tmem_ld_wait();
+          if (m < p.M) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              *reinterpret_cast<float4*>(prow + 32 * c + 4 * i) =
+                  make_float4(__uint_as_float(rr[4 * i]), __uint_as_float(rr[4 * i + 1]),
+                              __uint_as_float(rr[4 * i + 2]), __uint_as_float(rr[4 * i + 3]));
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&sh->sfreg_free[a]);
+          mbar_arrive(&sh->acc_empty[a]);
+        }
+        continue;
+      }
       uint32_t r[3][32];
 #pragma unroll
       for (int c = 0; c < 3; ++c) tmem_ld_x32(tmem + a * 256 + lane_off + 32 * c, r[c]);
@@ -392,6 +505,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
 
   tc_fence_before();
   __syncthreads();
+  if (S > 1) {
+    cluster_sync_all();  // every split's partial is in its CTA's shared memory
+    if (!sh->abort && tile0 < ntiles_total) split_reduce(p, part, split, tile0);
+    cluster_sync_relaxed();  // the peers have read this CTA's partial
+  }
   if (warp == 1) {
     if (lane == 0) wait_drain(&sh->done, 0, p.wait_ns);  // every MMA has retired
     __syncwarp();
@@ -411,6 +529,54 @@ int num_sms() {
   return n;
 }
 
+// Clusters of S CTAs of this kernel that fit on the device at once (cached
+// per device and S).
+int max_active_clusters(int S, size_t smem) {
+  static int cache[64][kMaxSplit + 1] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && cache[dev][S]) return cache[dev][S];
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(S, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = S;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_w4a4_kernel, &cfg) != cudaSuccess || n < 1) {
+    cudaGetLastError();
+    n = -1;  // cached as "does not fit"
+  }
+  if (dev >= 0 && dev < 64) cache[dev][S] = n;
+  return n;
+}
+
+// Split-K factor for `tiles` output tiles of `kt` K tiles plus `slab` low-rank
+// stages.  Splitting pays when the tiles leave most SMs idle: the time of a
+// tile is its longest split (the last split also runs the slab, one stage's
+// worth of MMAs each) plus about two K tiles for the reduction; every tile's
+// cluster must be resident at once.  Ties go to the smaller split.
+int choose_ksplit(int tiles, int kt, int slab, size_t smem) {
+  if (2 * tiles > num_sms()) return 1;
+  int best = 1;
+  long best_cost = kt + slab;
+  for (int S = 2; S <= std::min(kMaxSplit, kt); ++S) {
+    if (max_active_clusters(S, smem) < tiles) continue;
+    const int base = kt / S, rem = kt % S;
+    const long cost = std::max(base + (rem ? 1 : 0), base + slab) + 2;
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = S;
+    }
+  }
+  return best;
+}
+
 }  // namespace
 
 svdq_status launch_gemm_w4a4(const GemmArgs& a, cudaStream_t stream) {
@@ -425,6 +591,7 @@ svdq_status launch_gemm_w4a4(const GemmArgs& a, cudaStream_t stream) {
   p.slab = (a.r_pad + 31) / 32;
   p.mtiles = (a.M + 127) / 128;
   p.ntiles = (a.N + kBN - 1) / kBN;
+  p.ksplit = 1;
   p.xsf = static_cast<const uint8_t*>(a.xsf);
   p.wsf = a.wsf;
   p.bias = a.bias;
@@ -457,9 +624,28 @@ svdq_status launch_gemm_w4a4(const GemmArgs& a, cudaStream_t stream) {
     if (cur_dev >= 0 && cur_dev < 64) attr_set[cur_dev] = true;
   }
   const int tiles = p.mtiles * p.ntiles;
-  const int grid = std::min(tiles, num_sms());
-  gemm_w4a4_kernel<<<grid, kThreads, smem, stream>>>(map_xq, *a.map_wq_256, map_t, map_l2, p);
-  SVDQ_CUDA_TRY(cudaGetLastError());
+  if (a.ksplit > 0) {
+    p.ksplit = std::min(std::min(a.ksplit, kMaxSplit), p.kt);
+    if (p.ksplit > 1 && max_active_clusters(p.ksplit, smem) < tiles) p.ksplit = 1;
+  } else {
+    p.ksplit = choose_ksplit(tiles, p.kt, p.slab, smem);
+  }
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.ksplit > 1 ? tiles * p.ksplit : std::min(tiles, num_sms()), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = p.ksplit;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = p.ksplit > 1 ? 2 : 1;
+  SVDQ_CUDA_TRY(cudaLaunchKernelEx(&cfg, gemm_w4a4_kernel, map_xq, *a.map_wq_256, map_t, map_l2, p));
   return SVDQ_OK;
 }
 

@@ -72,7 +72,7 @@ struct GemmArgs {
   const float* bias;        // device [N]
   float alpha_w;
   void* Y;                  // device bf16 [M, N]
-  int force_bn;             // 0 = automatic, else 128 or 256
+  int ksplit;               // CTAs per output tile along K (0 = automatic, 1 = no split)
   int* err = nullptr;       // device error word (nullptr = the device's default word)
 };
 svdq_status launch_gemm_w4a4(const GemmArgs& a, cudaStream_t stream);
