@@ -61,10 +61,10 @@ def peaks():
 # kernel source the counters were taken on; counters of another source are stale
 # and not reported.
 K2_TRAFFIC = {
-    "source_sha256": "c33a1cc9f7370360dd404b28c33b271763f949f69845fa91e8d1da98a97dad2b",
+    "source_sha256": "fd419957ddb1a472fbbb8a953913cd3986f4fcd27e446f5a569aad328deeacb0",
     # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum: read + write per launch
-    "bytes_per_launch": {"attn_out": 14104064 + 11520, "qkv": 25144064 + 32850944,
-                         "mlp_up": 30659328 + 59751168, "mlp_down": 55489536 + 5601792},
+    "bytes_per_launch": {"attn_out": 14118656 + 1536, "qkv": 25145088 + 31958272,
+                         "mlp_up": 30719744 + 59113472, "mlp_down": 56924928 + 6905856},
 }
 
 

@@ -100,8 +100,16 @@ __device__ __noinline__ bool wait_drain(uint64_t* bar, uint32_t parity, uint64_t
   return true;
 }
 
-// y = alpha_w * acc + b for 32 consecutive columns of one row, bf16 RNE.  Each
-// lane writes whole 32-byte sectors when Y allows it (else 16-byte halves).
+// Two floats to a bf16x2 word (round to nearest even), the first in the low half.
+__device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// y = alpha_w * acc + b for 32 consecutive columns of one row, bf16 RNE.  alpha_w
+// is a power of two, so alpha_w * acc is exact (outside the subnormal range) and
+// one fused multiply-add rounds exactly like the product followed by the sum.
+// Each lane writes whole 32-byte sectors when Y allows it (else 16-byte halves).
 __device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], const float* bias_s, const K2Params& p,
                                             int m, int n) {
   if (m >= p.M || n >= p.N) return;
@@ -110,14 +118,12 @@ __device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], const float
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const float4 bv = b4[i];
-    const float y0 = __fadd_rn(__fmul_rn(__uint_as_float(r[4 * i + 0]), p.alpha_w), bv.x);
-    const float y1 = __fadd_rn(__fmul_rn(__uint_as_float(r[4 * i + 1]), p.alpha_w), bv.y);
-    const float y2 = __fadd_rn(__fmul_rn(__uint_as_float(r[4 * i + 2]), p.alpha_w), bv.z);
-    const float y3 = __fadd_rn(__fmul_rn(__uint_as_float(r[4 * i + 3]), p.alpha_w), bv.w);
-    packed[2 * i] = __bfloat16_as_ushort(__float2bfloat16_rn(y0)) |
-                    (uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(y1))) << 16);
-    packed[2 * i + 1] = __bfloat16_as_ushort(__float2bfloat16_rn(y2)) |
-                        (uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(y3))) << 16);
+    const float y0 = __fmaf_rn(__uint_as_float(r[4 * i + 0]), p.alpha_w, bv.x);
+    const float y1 = __fmaf_rn(__uint_as_float(r[4 * i + 1]), p.alpha_w, bv.y);
+    const float y2 = __fmaf_rn(__uint_as_float(r[4 * i + 2]), p.alpha_w, bv.z);
+    const float y3 = __fmaf_rn(__uint_as_float(r[4 * i + 3]), p.alpha_w, bv.w);
+    packed[2 * i] = bf16x2_rn(y0, y1);
+    packed[2 * i + 1] = bf16x2_rn(y2, y3);
   }
   uint16_t* dst = p.Y + static_cast<size_t>(m) * p.N + n;
   if (p.y32) {
@@ -160,14 +166,8 @@ __device__ __forceinline__ void split_reduce(const K2Params& p, const float* par
         acc.w = __fadd_rn(acc.w, v[q].w);
       }
     const float4 b = *reinterpret_cast<const float4*>(p.bias + n);
-    const float y0 = __fadd_rn(__fmul_rn(acc.x, p.alpha_w), b.x);
-    const float y1 = __fadd_rn(__fmul_rn(acc.y, p.alpha_w), b.y);
-    const float y2 = __fadd_rn(__fmul_rn(acc.z, p.alpha_w), b.z);
-    const float y3 = __fadd_rn(__fmul_rn(acc.w, p.alpha_w), b.w);
-    const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(y0)) |
-                        (uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(y1))) << 16);
-    const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(y2)) |
-                        (uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(y3))) << 16);
+    const uint32_t lo = bf16x2_rn(__fmaf_rn(acc.x, p.alpha_w, b.x), __fmaf_rn(acc.y, p.alpha_w, b.y));
+    const uint32_t hi = bf16x2_rn(__fmaf_rn(acc.z, p.alpha_w, b.z), __fmaf_rn(acc.w, p.alpha_w, b.w));
     *reinterpret_cast<uint2*>(p.Y + static_cast<size_t>(m0 + r) * p.N + n) = make_uint2(lo, hi);
   }
 }
