@@ -10,9 +10,10 @@ Modules:
   formats   E2M1 / E4M3 / bf16 encode and decode from their bit definitions
   codec     NVFP4 group-16 codec, nibble packing, block-scale atom layout
   svdquant  smoothing, SVD split, residual, weight factor, output, LoRA
+  int4      INT4 variant: group-64 codec with bf16 scales, nibble packing, output
 
 Parity status: every function is pinned by a CPU test against library casts,
 brute force, closed forms or invariants (tests/test_oracle_*.py).
 """
 
-from . import codec, formats, svdquant  # noqa: F401
+from . import codec, formats, int4, svdquant  # noqa: F401

@@ -193,3 +193,30 @@ def make_fp4_grid_inputs(M: int, K: int, N: int, seed: int,
     Xb, X = draw(M, x_exp)
     Wb, W = draw(N, w_exp)
     return Xb, X, Wb, W
+
+
+def make_int4_grid_inputs(M: int, K: int, N: int, seed: int,
+                          x_exp=(-2, 2), w_exp=(-9, -6), s_steps: int = 16):
+    """X [M,K] and W [N,K] whose every 64-element group along K is a set of
+    integers in -7..7 times a group scale s = 2^e (1 + j/s_steps), j <
+    s_steps (a power of two <= 16), with one element of each group at +-7 s,
+    so that amax / 7 = s exactly, s is a bf16 value and the group's INT4
+    encoding is exact.  Every value (at most 3 + 5 significant bits) is a bf16
+    value.  s_steps = 1 gives power-of-two scales.  Returns (X_bits, X, W_bits, W)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+
+    def draw(rows, exps):
+        q = rng.integers(-7, 8, size=(rows, K // 64, 64)).astype(np.float32)
+        pos = rng.integers(0, 64, size=(rows, K // 64))
+        sgn = rng.choice(np.array([-7.0, 7.0], np.float32), size=(rows, K // 64))
+        np.put_along_axis(q, pos[..., None], sgn[..., None], axis=-1)
+        e = rng.integers(exps[0], exps[1] + 1, size=(rows, K // 64, 1))
+        j = rng.integers(0, s_steps, size=(rows, K // 64, 1))
+        s = (np.ldexp(np.float32(1.0), e) * (1.0 + j / float(s_steps))).astype(np.float32)
+        v = (q * s).reshape(rows, K).astype(np.float32)
+        bits = f32_to_bf16_bits(v)
+        return bits, bf16_bits_to_f32(bits)
+
+    Xb, X = draw(M, x_exp)
+    Wb, W = draw(N, w_exp)
+    return Xb, X, Wb, W
