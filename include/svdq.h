@@ -63,6 +63,12 @@ typedef enum {
   SVDQ_ERR_DEVICE_CHECK = 6        /* a kernel's own bounds/launch check failed */
 } svdq_status;
 
+/* 4-bit format of the residual and the activations. */
+typedef enum {
+  SVDQ_FORMAT_NVFP4 = 0, /* E2M1 codes, E4M3 scale per 16 (App. D, Blackwell); the default */
+  SVDQ_FORMAT_INT4 = 1   /* signed INT4 codes (qmax 7, §3), bf16 scale per 64 (App. D "16-bit scales") */
+} svdq_format;
+
 /* Options of the offline weight transform. */
 typedef struct {
   float alpha;        /* smoothing migration strength (App. D); default 0.5 */
@@ -72,6 +78,7 @@ typedef struct {
   uint64_t seed;      /* seed of the random starting subspace; default 0 */
   int keep_residual;  /* nonzero: keep a host copy of R/alpha_w for export */
   int refine_iters;   /* splits tried (§4.2 refinement, see svdq_prepare_weights); default 1 */
+  int format;         /* svdq_format; default SVDQ_FORMAT_NVFP4 */
 } svdq_prepare_opts;
 
 /* Fills *opts with the defaults above. */
@@ -92,6 +99,10 @@ void svdq_prepare_opts_default(svdq_prepare_opts* opts);
  * L_{i+1} = SVD_r(W_hat - Q(W_hat - L_i)) for i < t, and the split whose
  * residual quantization error ||R - Q(R)||_F is smallest is kept
  * (svdq_weights_refine_errors reports the errors).
+ * With opts->format = SVDQ_FORMAT_INT4 the residual is coded in INT4 instead
+ * (groups of 64 along K, s = bf16(fp32(amax / 7)),
+ * q = clamp(rint(fp32(r_i * fp32(1/s))), -7, 7), round half to even, on the
+ * host; alpha_w = 1); refinement is NVFP4-only (refine_iters must be 1).
  *   W_bf16      host, N x K bf16 (out x in)
  *   act_absmax  host, K floats: per-input-channel max |x| over calibration data
  *   bias_bf16   host, N bf16, or NULL for no bias
@@ -149,6 +160,16 @@ svdq_status svdq_weights_from_factors(int N, int K, int rank, const float* inv_l
                                       const float* R, const float* bias, void* stream,
                                       svdq_weights** out);
 
+/* svdq_weights_from_factors with the residual's format chosen (svdq_format;
+ * SVDQ_FORMAT_INT4 codes R as svdq_prepare_weights describes). */
+svdq_status svdq_weights_from_factors_fmt(int N, int K, int rank, const float* inv_lam,
+                                          const uint16_t* L1p_bf16, const uint16_t* L2_bf16,
+                                          const float* R, const float* bias, int format, void* stream,
+                                          svdq_weights** out);
+
+/* The handle's svdq_format. */
+svdq_status svdq_weights_format(const svdq_weights* w, int* format);
+
 /*
  * LoRA without re-quantization (§2; §5.2 and Fig. 9: the low-rank branch
  * absorbs the LoRA by growing its rank).  Appends A as new columns of L1'
@@ -184,6 +205,13 @@ svdq_status svdq_quantize_act_lowrank_down(const svdq_weights* w, const void* X_
                                            void* xq, void* xsf, void* T, void* stream);
 
 /*
+ * For an INT4 handle the same call writes INT4 codes (two's-complement
+ * nibbles, element 2i in the low half of byte i) into xq and bf16 scales,
+ * group-major [K/64][round_up(M, 128)] with zeros for the padding rows, into
+ * xsf; the buffer sizes above cover both formats.
+ */
+
+/*
  * Kernel 2, the 4-bit GEMM with the up-projection folded in (§4.3):
  * Y = bf16_rne(alpha_w * (sum_k deq(xq) deq(wq) + (T_hi + T_lo) (L2 / alpha_w)) + b),
  * accumulated in fp32 in tensor memory.
@@ -196,6 +224,10 @@ svdq_status svdq_quantize_act_lowrank_down(const svdq_weights* w, const void* X_
  * fp32 accumulation error.  The launch is a programmatic dependent of the
  * kernel ahead of it in the stream: it reads xq, xsf and T only once that
  * kernel has completed.
+ * For an INT4 handle the codes and scales are expanded on chip into fp16 tiles
+ * (q * s with a bf16 s is exact in fp16 while |q s| stays in fp16's range)
+ * and contracted by fp16 tensor-core MMAs:
+ * Y = bf16_rne(sum_g s_x s_w sum_k q_x q_w + (T_hi + T_lo) L2 + b); no split-K.
  */
 svdq_status svdq_linear_w4a4(const svdq_weights* w, const void* xq, const void* xsf,
                              const void* T, int M, void* Y_bf16, void* stream);
@@ -253,6 +285,7 @@ size_t svdq_act_sf_bytes(int M, int K);                    /* ceil(M/128)*128 * 
 size_t svdq_lowrank_bytes(const svdq_weights* w, int M);   /* M * 2 * r_pad * 2 */
 size_t svdq_forward_workspace_bytes(const svdq_weights* w, int M);
 size_t svdq_forward_host_workspace_bytes(const svdq_weights* w, int M);
+size_t svdq_weights_sf_bytes(const svdq_weights* w);       /* the handle's weight scales */
 
 /* Shape of a handle: rank counts the SVD rank plus attached LoRA ranks, r_pad
  * is that rounded up to a multiple of 16 (the width of T's hi and lo parts). */
@@ -262,7 +295,9 @@ svdq_status svdq_weights_info(const svdq_weights* w, int* N, int* K, int* rank, 
 /*
  * Copies the handle's contents to host memory (tests and inspection).  Any
  * output may be NULL to skip it.
- *   codes     N x K/2 bytes        sf      svdq_act_sf_bytes(N, K) bytes (atom layout)
+ *   codes     N x K/2 bytes
+ *   sf        svdq_weights_sf_bytes(w) bytes: NVFP4 atom layout, or INT4 bf16
+ *             scales group-major [K/64][round_up(N, 256)]
  *   L1p_bf16  K x rank bf16        L2_bf16 rank x N bf16 (not divided by alpha_w)
  *   inv_lam   K floats             bias    N floats
  *   residual  N x K floats R/alpha_w; only if the handle kept it, else

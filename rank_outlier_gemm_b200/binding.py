@@ -33,7 +33,10 @@ class SvdqError(RuntimeError):
 class PrepareOpts(ctypes.Structure):
     _fields_ = [("alpha", ctypes.c_float), ("rank", ctypes.c_int), ("power_iters", ctypes.c_int),
                 ("oversample", ctypes.c_int), ("seed", ctypes.c_uint64), ("keep_residual", ctypes.c_int),
-                ("refine_iters", ctypes.c_int)]
+                ("refine_iters", ctypes.c_int), ("format", ctypes.c_int)]
+
+
+FORMATS = {"nvfp4": 0, "int4": 1}
 
 
 _vp, _i, _sz, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
@@ -41,6 +44,9 @@ _SIGS = {
     "svdq_prepare_opts_default": (None, [ctypes.POINTER(PrepareOpts)]),
     "svdq_prepare_weights": (_i, [_vp, _vp, _vp, _i, _i, ctypes.POINTER(PrepareOpts), _vp, ctypes.POINTER(_vp)]),
     "svdq_weights_from_factors": (_i, [_i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(_vp)]),
+    "svdq_weights_from_factors_fmt": (_i, [_i, _i, _i, _vp, _vp, _vp, _vp, _vp, _i, _vp, ctypes.POINTER(_vp)]),
+    "svdq_weights_format": (_i, [_vp, ctypes.POINTER(_i)]),
+    "svdq_weights_sf_bytes": (_sz, [_vp]),
     "svdq_attach_lora": (_i, [_vp, _vp, _vp, _i, _f, _vp]),
     "svdq_quantize_act_lowrank_down": (_i, [_vp, _vp, _i, _vp, _vp, _vp, _vp]),
     "svdq_linear_w4a4": (_i, [_vp, _vp, _vp, _vp, _i, _vp, _vp]),
@@ -135,7 +141,10 @@ class Weights:
         N, K, r, rp, aw = _i(), _i(), _i(), _i(), _f()
         _check(_lib.svdq_weights_info(self.handle, ctypes.byref(N), ctypes.byref(K), ctypes.byref(r),
                                       ctypes.byref(rp), ctypes.byref(aw)), "svdq_weights_info")
-        return {"N": N.value, "K": K.value, "rank": r.value, "r_pad": rp.value, "alpha_w": aw.value}
+        fmt = _i()
+        _check(_lib.svdq_weights_format(self.handle, ctypes.byref(fmt)), "svdq_weights_format")
+        return {"N": N.value, "K": K.value, "rank": r.value, "r_pad": rp.value, "alpha_w": aw.value,
+                "format": {v: k for k, v in FORMATS.items()}[fmt.value]}
 
     def __del__(self):
         if getattr(self, "handle", None):
@@ -151,7 +160,8 @@ def svdq_prepare_opts_default() -> PrepareOpts:
 
 def svdq_prepare_weights(W_bf16, act_absmax, bias_bf16=None, rank: int = 32, alpha: float = 0.5,
                          power_iters: int = 4, oversample: int = 16, seed: int = 0,
-                         keep_residual: bool = False, refine_iters: int = 1, stream=None) -> Weights:
+                         keep_residual: bool = False, refine_iters: int = 1, fmt: str = "nvfp4",
+                         stream=None) -> Weights:
     Wp, Wk = _host(W_bf16, np.uint16)
     N, K = Wk.shape
     ap, ak = _host(act_absmax, np.float32)
@@ -160,6 +170,7 @@ def svdq_prepare_weights(W_bf16, act_absmax, bias_bf16=None, rank: int = 32, alp
     o.alpha, o.rank, o.power_iters, o.oversample, o.seed = alpha, rank, power_iters, oversample, seed
     o.keep_residual = int(keep_residual)
     o.refine_iters = int(refine_iters)
+    o.format = FORMATS[fmt]
     h = _vp()
     _check(_lib.svdq_prepare_weights(Wp, ap, bp, N, K, ctypes.byref(o), _stream(stream), ctypes.byref(h)),
            "svdq_prepare_weights")
@@ -167,15 +178,15 @@ def svdq_prepare_weights(W_bf16, act_absmax, bias_bf16=None, rank: int = 32, alp
 
 
 def svdq_weights_from_factors(N: int, K: int, rank: int, inv_lam, L1p_bf16, L2_bf16, R, bias=None,
-                              stream=None) -> Weights:
+                              stream=None, fmt: str = "nvfp4") -> Weights:
     ip, ik = _host(inv_lam, np.float32)
     lp, lk = _host(L1p_bf16, np.uint16) if rank else (None, None)
     l2p, l2k = _host(L2_bf16, np.uint16) if rank else (None, None)
     rp, rk = _host(R, np.float32)
     bp, bk = _host(bias, np.float32)
     h = _vp()
-    _check(_lib.svdq_weights_from_factors(N, K, rank, ip, lp, l2p, rp, bp, _stream(stream), ctypes.byref(h)),
-           "svdq_weights_from_factors")
+    _check(_lib.svdq_weights_from_factors_fmt(N, K, rank, ip, lp, l2p, rp, bp, FORMATS[fmt], _stream(stream),
+                                              ctypes.byref(h)), "svdq_weights_from_factors_fmt")
     return Weights(h.value)
 
 
@@ -257,7 +268,7 @@ def svdq_weights_info(w: Weights) -> dict:
 def svdq_weights_export(w: Weights, residual: bool = False) -> dict:
     i = w.info
     N, K, r = i["N"], i["K"], i["rank"]
-    out = {"codes": np.empty((N, K // 2), np.uint8), "sf": np.empty(svdq_act_sf_bytes(N, K), np.uint8),
+    out = {"codes": np.empty((N, K // 2), np.uint8), "sf": np.empty(_lib.svdq_weights_sf_bytes(w.handle), np.uint8),
            "L1p": np.empty((K, r), np.uint16), "L2": np.empty((r, N), np.uint16),
            "inv_lam": np.empty(K, np.float32), "bias": np.empty(N, np.float32)}
     if residual:
@@ -275,7 +286,7 @@ def svdq_set_wait_limit_ns(ns: int) -> None:
 
 
 def svdq_search_alpha(W_bf16, X_bf16, bias_bf16=None, alphas=(0.3, 0.4, 0.5, 0.6, 0.7, 0.8), rank: int = 32,
-                      refine_iters: int = 1, stream=None):
+                      refine_iters: int = 1, fmt: str = "nvfp4", stream=None):
     """(relative output error per alpha, index of the best) on the calibration batch X."""
     Wp, Wk = _host(W_bf16, np.uint16)
     Xp, Xk = _host(X_bf16, np.uint16)
@@ -284,6 +295,7 @@ def svdq_search_alpha(W_bf16, X_bf16, bias_bf16=None, alphas=(0.3, 0.4, 0.5, 0.6
     a = np.ascontiguousarray(np.asarray(alphas, np.float32))
     o = svdq_prepare_opts_default()
     o.rank, o.refine_iters = rank, refine_iters
+    o.format = FORMATS[fmt]
     err = (ctypes.c_double * len(a))()
     best = ctypes.c_int(0)
     _check(_lib.svdq_search_alpha(Wp, Xp, Xk.shape[0], bp, N, K, a.ctypes.data, len(a), ctypes.byref(o),

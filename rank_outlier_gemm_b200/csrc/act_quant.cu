@@ -16,6 +16,12 @@
 // After the K loop the quantizer warps move T from TMEM to shared memory, the
 // cluster syncs, each CTA sums its share of rows over all S partials (fixed
 // order) and writes T as a bf16 hi/lo pair.
+//
+// The INT4 instantiation (SVDQuant App. D: groups of 64, 16-bit scales; §3:
+// qmax 7) quantizes each row's 64-column tile as one group: the lane pair
+// holding its two halves combines their maxima, s = bf16(fp32(amax / 7)),
+// q = clamp(rint(fp32(v * fp32(1 / s))), -7, 7), two's-complement nibbles,
+// and the bf16 scale goes to a group-major [K/64][rows padded to 128] array.
 #include <cooperative_groups.h>
 
 #include <algorithm>
@@ -46,6 +52,7 @@ struct K1Params {
   int* err;
   uint64_t wait_ns;
   int stall;
+  int m_pad;           // INT4: rows of the group-major scale array
   uint32_t l1_tile;    // r_pad * 128 bytes
   uint32_t tmem_cols;
 };
@@ -73,6 +80,18 @@ __device__ __forceinline__ void bar_sync_quant() {
   asm volatile("bar.sync 1, %0;" ::"n"(kQuantWarps * 32) : "memory");
 }
 
+// INT4: eight codes (element i in bits 4i..4i+3) of v[0..7] times r.
+__device__ __forceinline__ uint32_t int4x8(const float* v, float r) {
+  uint32_t w = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int q = min(7, max(-7, __float2int_rn(__fmul_rn(v[i], r))));
+    w |= (static_cast<uint32_t>(q) & 0xFu) << (4 * i);
+  }
+  return w;
+}
+
+template <bool kInt4>
 __global__ void __launch_bounds__(kThreads, 2) act_quant_lowrank_kernel(
     const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_l1,
     const K1Params p) {
@@ -182,26 +201,43 @@ __global__ void __launch_bounds__(kThreads, 2) act_quant_lowrank_kernel(
         v[8 * c + 0] = a0.x; v[8 * c + 1] = a0.y; v[8 * c + 2] = a1.x; v[8 * c + 3] = a1.y;
         v[8 * c + 4] = a2.x; v[8 * c + 5] = a2.y; v[8 * c + 6] = a3.x; v[8 * c + 7] = a3.y;
       }
-      float g0[16], g1[16];
+      if constexpr (kInt4) {
+        float amax = 0.0f;
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        g0[j] = v[j];
-        g1[j] = v[16 + j];
-      }
-      const Fp4Group q0 = nvfp4_encode16(g0, sh->rcp_tbl);
-      const Fp4Group q1 = nvfp4_encode16(g1, sh->rcp_tbl);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sh->empty[s]);  // this warp is done reading the stage
-      if (m < p.M) {
-        uint4* dst = reinterpret_cast<uint4*>(p.xq + static_cast<size_t>(m) * (p.K / 2) + k0 / 2 + 16 * h);
-        *dst = make_uint4(q0.lo, q0.hi, q1.lo, q1.hi);
-      }
-      const uint32_t mine = q0.scale | (q1.scale << 8);
-      const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
-      if (h == 0) {
-        const size_t atom = static_cast<size_t>(mb) * p.kt_total + kt;
-        *reinterpret_cast<uint32_t*>(p.xsf + atom * 512 + (row & 31) * 16 + (row >> 5) * 4) =
-            mine | (other << 16);
+        for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(v[j]));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));  // the other half of the group
+        const __nv_bfloat16 sb = __float2bfloat16_rn(__fdiv_rn(amax, 7.0f));
+        const float sv = __bfloat162float(sb);
+        const float r = sv > 0.0f ? __frcp_rn(sv) : 0.0f;
+        const uint4 codes = make_uint4(int4x8(v, r), int4x8(v + 8, r), int4x8(v + 16, r), int4x8(v + 24, r));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh->empty[s]);  // this warp is done reading the stage
+        if (m < p.M)
+          *reinterpret_cast<uint4*>(p.xq + static_cast<size_t>(m) * (p.K / 2) + k0 / 2 + 16 * h) = codes;
+        if (h == 0)
+          reinterpret_cast<uint16_t*>(p.xsf)[static_cast<size_t>(kt) * p.m_pad + m] = __bfloat16_as_ushort(sb);
+      } else {
+        float g0[16], g1[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          g0[j] = v[j];
+          g1[j] = v[16 + j];
+        }
+        const Fp4Group q0 = nvfp4_encode16(g0, sh->rcp_tbl);
+        const Fp4Group q1 = nvfp4_encode16(g1, sh->rcp_tbl);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh->empty[s]);  // this warp is done reading the stage
+        if (m < p.M) {
+          uint4* dst = reinterpret_cast<uint4*>(p.xq + static_cast<size_t>(m) * (p.K / 2) + k0 / 2 + 16 * h);
+          *dst = make_uint4(q0.lo, q0.hi, q1.lo, q1.hi);
+        }
+        const uint32_t mine = q0.scale | (q1.scale << 8);
+        const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
+        if (h == 0) {
+          const size_t atom = static_cast<size_t>(mb) * p.kt_total + kt;
+          *reinterpret_cast<uint32_t*>(p.xsf + atom * 512 + (row & 31) * 16 + (row >> 5) * 4) =
+              mine | (other << 16);
+        }
       }
     }
     if (lowrank) {
@@ -285,13 +321,13 @@ __global__ void __launch_bounds__(kThreads, 2) act_quant_lowrank_kernel(
 
 // Clusters of this kernel that fit on the device at once for a K-split of S
 // (cluster = S CTAs); cached per (S, shared memory size).
-int max_active_clusters(int S, size_t smem) {
+int max_active_clusters(int S, size_t smem, bool int4) {
   static std::mutex mu;
   static std::map<std::pair<int, size_t>, int> cache;
   std::lock_guard<std::mutex> lk(mu);
   int dev = 0;
   cudaGetDevice(&dev);
-  const auto key = std::make_pair(S + 16 * dev, smem);
+  const auto key = std::make_pair(S + 16 * dev + (int4 ? 4096 : 0), smem);
   auto it = cache.find(key);
   if (it != cache.end()) return it->second;
   cudaLaunchConfig_t cfg = {};
@@ -306,7 +342,9 @@ int max_active_clusters(int S, size_t smem) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, act_quant_lowrank_kernel, &cfg) != cudaSuccess || n < 1) {
+  const cudaError_t qe = int4 ? cudaOccupancyMaxActiveClusters(&n, act_quant_lowrank_kernel<true>, &cfg)
+                              : cudaOccupancyMaxActiveClusters(&n, act_quant_lowrank_kernel<false>, &cfg);
+  if (qe != cudaSuccess || n < 1) {
     cudaGetLastError();
     n = 1;
   }
@@ -319,12 +357,12 @@ int max_active_clusters(int S, size_t smem) {
 // placed one CTA per SM within a GPC, so splitting more only pays while the
 // clusters still fit: the cost is (waves of clusters) x (tiles per CTA), ties
 // going to the larger split (more CTAs in flight).  At least 4 tiles per CTA.
-int auto_splits(int mblocks, int kt_total, size_t smem) {
+int auto_splits(int mblocks, int kt_total, size_t smem, bool int4) {
   const int s_max = std::max(1, std::min(8, kt_total / 4));
   int best = 1;
   long best_cost = -1;
   for (int S = 1; S <= s_max; ++S) {
-    const int fit = max_active_clusters(S, smem);
+    const int fit = max_active_clusters(S, smem, int4);
     const long waves = (mblocks + fit - 1) / fit;
     const long cost = waves * ((kt_total + S - 1) / S);
     if (best_cost < 0 || cost <= best_cost) {
@@ -346,11 +384,12 @@ svdq_status launch_act_quant(const ActArgs& a, cudaStream_t stream) {
   int cur_dev = 0;
   SVDQ_CUDA_TRY(cudaGetDevice(&cur_dev));
   if (cur_dev < 0 || cur_dev >= 64 || !attr_set[cur_dev]) {
-    SVDQ_CUDA_TRY(cudaFuncSetAttribute(act_quant_lowrank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024));
+    SVDQ_CUDA_TRY(cudaFuncSetAttribute(act_quant_lowrank_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024));
+    SVDQ_CUDA_TRY(cudaFuncSetAttribute(act_quant_lowrank_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024));
     if (cur_dev >= 0 && cur_dev < 64) attr_set[cur_dev] = true;
   }
   const int splits = a.splits > 0 ? std::min(std::min(a.splits, 8), kt_total)
-                                   : auto_splits(mblocks, kt_total, smem);
+                                   : auto_splits(mblocks, kt_total, smem, a.int4 != 0);
 
   CUtensorMap map_x;
   svdq_status st = make_tmap_2d(&map_x, a.X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.K, a.M,
@@ -371,6 +410,7 @@ svdq_status launch_act_quant(const ActArgs& a, cudaStream_t stream) {
   p.err = a.err ? a.err : device_error_word();
   p.wait_ns = wait_limit_ns();
   p.stall = a.stall;
+  p.m_pad = mblocks * 128;
   p.l1_tile = l1_tile;
   uint32_t cols = 32;
   while (cols < static_cast<uint32_t>(a.r_pad)) cols <<= 1;
@@ -389,7 +429,10 @@ svdq_status launch_act_quant(const ActArgs& a, cudaStream_t stream) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  SVDQ_CUDA_TRY(cudaLaunchKernelEx(&cfg, act_quant_lowrank_kernel, map_x, map_l1, p));
+  if (a.int4)
+    SVDQ_CUDA_TRY(cudaLaunchKernelEx(&cfg, act_quant_lowrank_kernel<true>, map_x, map_l1, p));
+  else
+    SVDQ_CUDA_TRY(cudaLaunchKernelEx(&cfg, act_quant_lowrank_kernel<false>, map_x, map_l1, p));
   return SVDQ_OK;
 }
 

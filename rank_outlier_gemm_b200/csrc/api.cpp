@@ -148,7 +148,7 @@ svdq_status upload_lowrank(svdq_weights* w, cudaStream_t stream) {
 }
 
 svdq_status build_handle(int N, int K, int rank, const float* inv_lam, const uint16_t* L1p,
-                         const uint16_t* L2, const float* R, const float* bias, int keep_residual,
+                         const uint16_t* L2, const float* R, const float* bias, int keep_residual, int format,
                          cudaStream_t stream, svdq_weights** out) {
   svdq_weights* w = new (std::nothrow) svdq_weights();
   if (!w) return fail(SVDQ_ERR_OOM, "host allocation failed");
@@ -161,8 +161,10 @@ svdq_status build_handle(int N, int K, int rank, const float* inv_lam, const uin
   w->N = N;
   w->K = K;
   w->rank = rank;
+  w->format = format;
   const size_t nk = static_cast<size_t>(N) * K;
-  w->alpha_w = weight_factor(R, nk);
+  // INT4's bf16 scales span fp32's exponent range: no per-tensor factor
+  w->alpha_w = format == SVDQ_FORMAT_INT4 ? 1.0f : weight_factor(R, nk);
   w->inv_lam.assign(inv_lam, inv_lam + K);
   if (rank > 0) {
     w->L1p.assign(L1p, L1p + static_cast<size_t>(K) * rank);
@@ -174,8 +176,9 @@ svdq_status build_handle(int N, int K, int rank, const float* inv_lam, const uin
   for (size_t i = 0; i < nk; ++i) Rp[i] = static_cast<float>(static_cast<double>(R[i]) / w->alpha_w);
   if (keep_residual) w->residual = Rp;
 
-  const int npad = round_up(N, 128);
-  const size_t sf_bytes = static_cast<size_t>(npad) * (K / 16);
+  const int npad = format == SVDQ_FORMAT_INT4 ? round_up(N, 256) : round_up(N, 128);
+  const size_t sf_bytes = format == SVDQ_FORMAT_INT4 ? static_cast<size_t>(K / 64) * npad * 2
+                                                      : static_cast<size_t>(npad) * (K / 16);
   cudaError_t e;
   if ((e = cudaMalloc(&w->d_wq, nk / 2)) != cudaSuccess) return bail(cuda_fail(e, "cudaMalloc codes"));
   if ((e = cudaMalloc(&w->d_wsf, sf_bytes)) != cudaSuccess) return bail(cuda_fail(e, "cudaMalloc scales"));
@@ -188,7 +191,22 @@ svdq_status build_handle(int N, int K, int rank, const float* inv_lam, const uin
   float* d_R = nullptr;
   if ((e = cudaMalloc(&d_R, nk * 4)) != cudaSuccess) return bail(cuda_fail(e, "cudaMalloc residual"));
   svdq_status st = SVDQ_OK;
+  std::vector<uint8_t> h_codes;
+  std::vector<uint16_t> h_scales;
+  if (format == SVDQ_FORMAT_INT4) {  // offline host codec; the device gets packed codes and scales
+    h_codes.assign(nk / 2, 0);
+    h_scales.assign(sf_bytes / 2, 0);
+    int4_encode_rows(Rp.data(), N, K, npad, h_codes.data(), h_scales.data());
+  }
   do {
+    if (format == SVDQ_FORMAT_INT4) {
+      if ((e = cudaMemcpyAsync(w->d_wq, h_codes.data(), nk / 2, cudaMemcpyHostToDevice, stream)) != cudaSuccess ||
+          (e = cudaMemcpyAsync(w->d_wsf, h_scales.data(), sf_bytes, cudaMemcpyHostToDevice, stream)) !=
+              cudaSuccess) {
+        st = cuda_fail(e, "cudaMemcpyAsync INT4 codes");
+        break;
+      }
+    }
     if ((e = cudaMemcpyAsync(d_R, Rp.data(), nk * 4, cudaMemcpyHostToDevice, stream)) != cudaSuccess ||
         (e = cudaMemcpyAsync(w->d_inv_lam, inv_lam, static_cast<size_t>(K) * 4, cudaMemcpyHostToDevice,
                              stream)) != cudaSuccess ||
@@ -197,14 +215,23 @@ svdq_status build_handle(int N, int K, int rank, const float* inv_lam, const uin
       st = cuda_fail(e, "cudaMemcpyAsync weights");
       break;
     }
-    st = launch_weight_codec(d_R, N, K, w->d_wq, w->d_wsf, stream);
-    if (st != SVDQ_OK) break;
+    if (format != SVDQ_FORMAT_INT4) {
+      st = launch_weight_codec(d_R, N, K, w->d_wq, w->d_wsf, stream);
+      if (st != SVDQ_OK) break;
+    }
     if ((e = cudaStreamSynchronize(stream)) != cudaSuccess) st = cuda_fail(e, "weight codec");
   } while (0);
   cudaFree(d_R);
   if (st != SVDQ_OK) return bail(st);
   st = upload_lowrank(w, stream);
   if (st != SVDQ_OK) return bail(st);
+  if (format == SVDQ_FORMAT_INT4) {  // one 64-wide group (32 bytes) of 256 rows per load
+    st = make_tmap_2d(&w->map_wq_256, w->d_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, N, K / 2, 32, 256,
+                      CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != SVDQ_OK) return bail(st);
+    *out = w;
+    return SVDQ_OK;
+  }
   st = make_tmap_2d(&w->map_wq_256, w->d_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, N, K / 2, 128, 256,
                     CU_TENSOR_MAP_SWIZZLE_128B);
   if (st == SVDQ_OK)
@@ -292,6 +319,7 @@ void svdq_prepare_opts_default(svdq_prepare_opts* o) {
   o->seed = 0;
   o->keep_residual = 0;
   o->refine_iters = 1;
+  o->format = SVDQ_FORMAT_NVFP4;
 }
 
 svdq_status svdq_prepare_weights(const uint16_t* W_bf16, const float* act_absmax, const uint16_t* bias_bf16,
@@ -309,6 +337,10 @@ svdq_status svdq_prepare_weights(const uint16_t* W_bf16, const float* act_absmax
   if (!(o.alpha >= 0.0f && o.alpha <= 1.0f)) return fail(SVDQ_ERR_INVALID_ARG, "alpha must be in [0, 1]");
   if (o.refine_iters < 1 || o.refine_iters > 64)
     return fail(SVDQ_ERR_INVALID_ARG, "refine_iters=%d must be in [1, 64]", o.refine_iters);
+  if (o.format != SVDQ_FORMAT_NVFP4 && o.format != SVDQ_FORMAT_INT4)
+    return fail(SVDQ_ERR_INVALID_ARG, "format=%d is neither NVFP4 (0) nor INT4 (1)", o.format);
+  if (o.format == SVDQ_FORMAT_INT4 && o.refine_iters != 1)
+    return fail(SVDQ_ERR_INVALID_ARG, "refinement (refine_iters > 1) is implemented for NVFP4 only");
   for (int k = 0; k < K; ++k)
     if (!std::isfinite(act_absmax[k]) || act_absmax[k] < 0)
       return fail(SVDQ_ERR_INVALID_ARG, "act_absmax[%d] is negative or not finite", k);
@@ -321,8 +353,8 @@ svdq_status svdq_prepare_weights(const uint16_t* W_bf16, const float* act_absmax
     for (int n = 0; n < N; ++n) bias[n] = bf16_to_f32(bias_bf16[n]);
   }
   SVDQ_TRY(build_handle(N, K, o.rank, hs.inv_lam.data(), hs.L1p.data(), hs.L2.data(), hs.R.data(),
-                        bias_bf16 ? bias.data() : nullptr, o.keep_residual, static_cast<cudaStream_t>(stream),
-                        out));
+                        bias_bf16 ? bias.data() : nullptr, o.keep_residual, o.format,
+                        static_cast<cudaStream_t>(stream), out));
   (*out)->refine_err = hs.refine_err;
   return SVDQ_OK;
 }
@@ -350,7 +382,41 @@ svdq_status svdq_weights_from_factors(int N, int K, int rank, const float* inv_l
   for (int k = 0; k < K; ++k)
     if (!std::isfinite(inv_lam[k])) return fail(SVDQ_ERR_INVALID_ARG, "inv_lam has a non-finite value");
   SVDQ_TRY(check_device());
-  return build_handle(N, K, rank, inv_lam, L1p_bf16, L2_bf16, R, bias, 1, static_cast<cudaStream_t>(stream), out);
+  return build_handle(N, K, rank, inv_lam, L1p_bf16, L2_bf16, R, bias, 1, SVDQ_FORMAT_NVFP4,
+                      static_cast<cudaStream_t>(stream), out);
+}
+
+svdq_status svdq_weights_from_factors_fmt(int N, int K, int rank, const float* inv_lam, const uint16_t* L1p_bf16,
+                                          const uint16_t* L2_bf16, const float* R, const float* bias, int format,
+                                          void* stream, svdq_weights** out) {
+  if (format != SVDQ_FORMAT_NVFP4 && format != SVDQ_FORMAT_INT4)
+    return fail(SVDQ_ERR_INVALID_ARG, "format=%d is neither NVFP4 (0) nor INT4 (1)", format);
+  if (format == SVDQ_FORMAT_NVFP4)
+    return svdq_weights_from_factors(N, K, rank, inv_lam, L1p_bf16, L2_bf16, R, bias, stream, out);
+  if (!out) return fail(SVDQ_ERR_INVALID_ARG, "out is null");
+  *out = nullptr;
+  SVDQ_TRY(check_shape(N, K));
+  if (rank < 0 || rank > 128) return fail(SVDQ_ERR_INVALID_ARG, "rank=%d must be in [0, 128]", rank);
+  if (!inv_lam || !R) return fail(SVDQ_ERR_INVALID_ARG, "inv_lam and R are required");
+  if (rank > 0 && (!L1p_bf16 || !L2_bf16)) return fail(SVDQ_ERR_INVALID_ARG, "rank > 0 needs L1p and L2");
+  const size_t nk = static_cast<size_t>(N) * K;
+  for (size_t i = 0; i < nk; ++i)
+    if (!std::isfinite(R[i])) return fail(SVDQ_ERR_INVALID_ARG, "R has a non-finite value");
+  SVDQ_TRY(check_device());
+  return build_handle(N, K, rank, inv_lam, L1p_bf16, L2_bf16, R, bias, 1, format, static_cast<cudaStream_t>(stream),
+                      out);
+}
+
+svdq_status svdq_weights_format(const svdq_weights* w, int* format) {
+  if (!w || !format) return fail(SVDQ_ERR_INVALID_ARG, "null weights handle or format");
+  *format = w->format;
+  return SVDQ_OK;
+}
+
+size_t svdq_weights_sf_bytes(const svdq_weights* w) {
+  if (!w) return 0;
+  return w->format == SVDQ_FORMAT_INT4 ? static_cast<size_t>(w->K / 64) * round_up(w->N, 256) * 2
+                                       : svdq_act_sf_bytes(w->N, w->K);
 }
 
 svdq_status svdq_attach_lora(svdq_weights* w, const uint16_t* A_bf16, const uint16_t* B_bf16, int r_l,
@@ -387,6 +453,7 @@ svdq_status svdq_quantize_act_lowrank_down(const svdq_weights* w, const void* X_
   if (w->r_pad > 0) SVDQ_TRY(check_dev_ptr(T, "T"));
   ActArgs a{M, w->K, w->r_pad, X_bf16, &w->map_l1, w->d_inv_lam, static_cast<uint8_t*>(xq),
             static_cast<uint8_t*>(xsf), static_cast<uint16_t*>(T), 0, 0};
+  a.int4 = w->format == SVDQ_FORMAT_INT4;
   return launch_act_quant(a, static_cast<cudaStream_t>(stream));
 }
 
@@ -399,6 +466,7 @@ svdq_status svdq_debug_launch_stalled_act(const svdq_weights* w, const void* X_b
   if (w->r_pad > 0) SVDQ_TRY(check_dev_ptr(T, "T"));
   ActArgs a{M, w->K, w->r_pad, X_bf16, &w->map_l1, w->d_inv_lam, static_cast<uint8_t*>(xq),
             static_cast<uint8_t*>(xsf), static_cast<uint16_t*>(T), 1, 0};
+  a.int4 = w->format == SVDQ_FORMAT_INT4;
   return launch_act_quant(a, static_cast<cudaStream_t>(stream));
 }
 
@@ -408,6 +476,15 @@ svdq_status svdq_selftest_codec(unsigned int* mismatches) {
   return selftest_codec(mismatches);
 }
 
+namespace {
+svdq_status launch_int4(const svdq_weights* w, const void* xq, const void* xsf, const void* T, int M, void* Y,
+                        void* stream) {
+  GemmInt4Args a{M, w->N, w->K, w->r_pad, xq, xsf, T, &w->map_wq_256, &w->map_l2_256,
+                 reinterpret_cast<const uint16_t*>(w->d_wsf), w->d_bias, Y};
+  return launch_gemm_int4(a, static_cast<cudaStream_t>(stream));
+}
+}  // namespace
+
 svdq_status svdq_linear_w4a4(const svdq_weights* w, const void* xq, const void* xsf, const void* T, int M,
                              void* Y_bf16, void* stream) {
   SVDQ_TRY(check_runtime(w, M));
@@ -415,6 +492,7 @@ svdq_status svdq_linear_w4a4(const svdq_weights* w, const void* xq, const void* 
   SVDQ_TRY(check_dev_ptr(xsf, "xsf"));
   SVDQ_TRY(check_dev_ptr(Y_bf16, "Y"));
   if (w->r_pad > 0) SVDQ_TRY(check_dev_ptr(T, "T"));
+  if (w->format == SVDQ_FORMAT_INT4) return launch_int4(w, xq, xsf, T, M, Y_bf16, stream);
   GemmArgs a{M, w->N, w->K, w->r_pad, xq, xsf, T, &w->map_wq_256, &w->map_wq_128, &w->map_l2_256,
              &w->map_l2_128, w->d_wsf, w->d_bias, w->alpha_w, Y_bf16, 0};
   return launch_gemm_w4a4(a, static_cast<cudaStream_t>(stream));
@@ -428,6 +506,7 @@ svdq_status svdq_debug_linear_w4a4_ksplit(const svdq_weights* w, const void* xq,
   SVDQ_TRY(check_dev_ptr(xsf, "xsf"));
   SVDQ_TRY(check_dev_ptr(Y_bf16, "Y"));
   if (w->r_pad > 0) SVDQ_TRY(check_dev_ptr(T, "T"));
+  if (w->format == SVDQ_FORMAT_INT4) return launch_int4(w, xq, xsf, T, M, Y_bf16, stream);  // no split-K
   GemmArgs a{M, w->N, w->K, w->r_pad, xq, xsf, T, &w->map_wq_256, &w->map_wq_128, &w->map_l2_256,
              &w->map_l2_128, w->d_wsf, w->d_bias, w->alpha_w, Y_bf16, ksplit};
   return launch_gemm_w4a4(a, static_cast<cudaStream_t>(stream));
@@ -535,7 +614,7 @@ svdq_status svdq_weights_export(const svdq_weights* w, uint8_t* codes, uint8_t* 
   if (residual && w->residual.empty()) return fail(SVDQ_ERR_INVALID_ARG, "the handle kept no residual");
   SVDQ_CUDA_TRY(cudaDeviceSynchronize());
   if (codes) SVDQ_CUDA_TRY(cudaMemcpy(codes, w->d_wq, static_cast<size_t>(w->N) * w->K / 2, cudaMemcpyDeviceToHost));
-  if (sf) SVDQ_CUDA_TRY(cudaMemcpy(sf, w->d_wsf, svdq_act_sf_bytes(w->N, w->K), cudaMemcpyDeviceToHost));
+  if (sf) SVDQ_CUDA_TRY(cudaMemcpy(sf, w->d_wsf, svdq_weights_sf_bytes(w), cudaMemcpyDeviceToHost));
   if (L1p_bf16) std::copy(w->L1p.begin(), w->L1p.end(), L1p_bf16);
   if (L2_bf16) std::copy(w->L2.begin(), w->L2.end(), L2_bf16);
   if (inv_lam) std::copy(w->inv_lam.begin(), w->inv_lam.end(), inv_lam);

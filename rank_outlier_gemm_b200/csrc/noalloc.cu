@@ -82,8 +82,15 @@ extern "C" svdq_status svdq_forward_noalloc(const svdq_weights* w, const void* X
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   ActArgs a{M, w->K, w->r_pad, X_bf16, &w->map_l1, w->d_inv_lam, xq, xsf, T, 0, 0};
   a.err = d.err;
+  a.int4 = w->format == SVDQ_FORMAT_INT4;
   st = launch_act_quant(a, s);
   if (st != SVDQ_OK) return st;
+  if (w->format == SVDQ_FORMAT_INT4) {
+    GemmInt4Args g{M, w->N, w->K, w->r_pad, xq, xsf, T, &w->map_wq_256, &w->map_l2_256,
+                   reinterpret_cast<const uint16_t*>(w->d_wsf), w->d_bias, Y_bf16};
+    g.err = d.err;
+    return launch_gemm_int4(g, s);
+  }
   GemmArgs g{M, w->N, w->K, w->r_pad, xq, xsf, T, &w->map_wq_256, &w->map_wq_128, &w->map_l2_256,
              &w->map_l2_128, w->d_wsf, w->d_bias, w->alpha_w, Y_bf16, 0};
   g.err = d.err;

@@ -55,6 +55,35 @@ float weight_factor(const float* R, size_t n) {
   return static_cast<float>(std::ldexp(1.0, c));
 }
 
+// INT4 codec (SVDQuant App. D: groups of 64 with 16-bit scales; §3: qmax 7):
+// s = bf16(fp32(amax / 7)), q = clamp(rint(fp32(v * fp32(1 / s))), -7, 7) with
+// round-half-even, two's-complement nibbles with element 2i in the low half
+// of byte i.  IEEE fp32 host arithmetic (no contraction across the steps).
+void int4_encode_rows(const float* R, int rows, int K, int rows_pad, uint8_t* codes, uint16_t* scales) {
+  const int G = K / 64;
+  for (int n = 0; n < rows; ++n) {
+    const float* v = R + static_cast<size_t>(n) * K;
+    uint8_t* c = codes + static_cast<size_t>(n) * (K / 2);
+    for (int g = 0; g < G; ++g) {
+      float amax = 0.0f;
+      for (int j = 0; j < 64; ++j) amax = std::max(amax, std::fabs(v[64 * g + j]));
+      volatile float q7 = amax / 7.0f;  // one fp32 rounding before the bf16 one
+      const uint16_t sb = f32_to_bf16_rne(q7);
+      scales[static_cast<size_t>(g) * rows_pad + n] = sb;
+      const float sv = bf16_to_f32(sb);
+      volatile float r = sv > 0.0f ? 1.0f / sv : 0.0f;
+      for (int j = 0; j < 64; j += 2) {
+        int q[2];
+        for (int e = 0; e < 2; ++e) {
+          volatile float t = v[64 * g + j + e] * r;
+          q[e] = std::min(7, std::max(-7, static_cast<int>(std::nearbyint(t))));
+        }
+        c[32 * g + j / 2] = static_cast<uint8_t>((q[0] & 0xF) | ((q[1] & 0xF) << 4));
+      }
+    }
+  }
+}
+
 namespace {
 
 void parallel_for(long n, const std::function<void(long, long)>& body) {

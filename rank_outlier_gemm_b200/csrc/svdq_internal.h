@@ -56,6 +56,7 @@ struct ActArgs {
   int stall;                // test hook: a wait that never completes
   int splits;               // K-splits per 128-row block (0 = automatic)
   int* err = nullptr;       // device error word (nullptr = the device's default word)
+  int int4 = 0;             // INT4 variant: group-64 codes, bf16 scales [K/64][rows padded to 128]
 };
 svdq_status launch_act_quant(const ActArgs& a, cudaStream_t stream);
 
@@ -76,6 +77,24 @@ struct GemmArgs {
   int* err = nullptr;       // device error word (nullptr = the device's default word)
 };
 svdq_status launch_gemm_w4a4(const GemmArgs& a, cudaStream_t stream);
+
+struct GemmInt4Args {
+  int M, N, K, r_pad;
+  const void* xq;           // device [M, K/2] packed INT4
+  const void* xsf;          // device bf16 [K/64][round_up(M, 128)]
+  const void* T;            // device [M, 2 r_pad] bf16
+  const CUtensorMap* map_wq;      // weight codes [N, K/2], box 32 bytes x 256 rows
+  const CUtensorMap* map_l2_256;  // L2^T [N, r_pad] bf16, box rows 256
+  const uint16_t* wsf;      // device bf16 [K/64][round_up(N, 256)]
+  const float* bias;        // device [round_up(N, 256)]
+  void* Y;                  // device bf16 [M, N]
+  int* err = nullptr;
+};
+svdq_status launch_gemm_int4(const GemmInt4Args& a, cudaStream_t stream);
+
+// INT4 codec of fp32 rows [rows, K] (host, offline): packed codes [rows, K/2]
+// and bf16 scales group-major [K/64][rows_pad] (padded rows left untouched).
+void int4_encode_rows(const float* R, int rows, int K, int rows_pad, uint8_t* codes, uint16_t* scales);
 
 // Device self-test of the encoder's exact division and reciprocal shortcuts.
 svdq_status selftest_codec(unsigned int* mismatches_out);
@@ -104,12 +123,14 @@ float weight_factor(const float* R, size_t n);
 // The opaque handle.
 struct svdq_weights {
   int device = 0;
+  int format = 0;     // SVDQ_FORMAT_NVFP4 or SVDQ_FORMAT_INT4
   int N = 0, K = 0;
   int rank = 0;       // SVD rank + LoRA ranks
   int r_pad = 0;      // rank rounded up to 16
   float alpha_w = 1.0f;
   uint8_t* d_wq = nullptr;       // [N, K/2]
-  uint8_t* d_wsf = nullptr;      // [ceil(N/128)*128, K/16] atom layout
+  uint8_t* d_wsf = nullptr;      // NVFP4: [ceil(N/128)*128, K/16] atom layout;
+                                 // INT4: bf16 [K/64][round_up(N, 256)]
   float* d_inv_lam = nullptr;    // [K]
   uint16_t* d_L1t = nullptr;     // [r_pad, K] bf16 = L1'^T
   uint16_t* d_L2t = nullptr;     // [N, r_pad] bf16 = L2^T / alpha_w

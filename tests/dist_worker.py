@@ -22,8 +22,9 @@ def main():
     slowest = bench.max_over_ranks(mine, world, torch.device("cpu"))
     value = bench.job_throughput(1e9, slowest, world)
     dist.barrier()
-    print(json.dumps({"rank": rank, "world": world, "local": local, "mine": mine, "slowest": slowest,
-                      "value": value}), flush=True)
+    line = json.dumps({"rank": rank, "world": world, "local": local, "mine": mine, "slowest": slowest,
+                       "value": value}) + "\n"
+    os.write(1, line.encode())  # one write: the ranks share the pipe, lines must not interleave
     dist.destroy_process_group()
 
 

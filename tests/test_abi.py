@@ -40,6 +40,7 @@ def test_host_only_helpers():
     assert B.svdq_act_sf_bytes(129, 64) == 256 * 4
     o = B.svdq_prepare_opts_default()
     assert (o.alpha, o.rank, o.power_iters, o.oversample, o.refine_iters) == (0.5, 32, 4, 16, 1)
+    assert o.format == B.FORMATS["nvfp4"] == 0 and B.FORMATS["int4"] == 1
     assert "sm_100a" in B.svdq_version()
 
 
@@ -60,6 +61,15 @@ def test_invalid_arguments_rejected_before_gpu():
     with pytest.raises(B.SvdqError) as e:   # refinement needs at least one split
         B.svdq_prepare_weights(W, np.ones(64, np.float32), rank=4, refine_iters=0)
     assert e.value.status == 1 and "refine_iters" in str(e.value)
+    with pytest.raises(B.SvdqError) as e:   # refinement is NVFP4-only
+        B.svdq_prepare_weights(W, np.ones(64, np.float32), rank=4, fmt="int4", refine_iters=2)
+    assert e.value.status == 1 and "NVFP4 only" in str(e.value)
+    import ctypes
+    h = ctypes.c_void_p()
+    R0 = np.zeros((32, 64), np.float32)
+    st = B._lib.svdq_weights_from_factors_fmt(32, 64, 0, np.ones(64, np.float32).ctypes.data, None, None,
+                                              R0.ctypes.data, None, 7, None, ctypes.byref(h))
+    assert st == 1 and b"format" in B._lib.svdq_last_error()
     bad = np.ones(64, np.float32)
     bad[3] = np.nan
     with pytest.raises(B.SvdqError) as e:
