@@ -301,6 +301,34 @@ def refinement(L, iters=4):
     return out
 
 
+def int4_layers(L, torch, layers, dev, stream, reps=30):
+    """NEXT-4, the INT4 variant (App. D: groups of 64, 16-bit scales) on the step's
+    layers: library-prepared INT4 weights (rank 32), layer time (both kernels)
+    and GEMM time, the GEMM's rate against the measured dense bf16 peak (its
+    contraction runs on fp16 tiles dequantized on chip), and the NVFP4 layer
+    time for comparison."""
+    pk = peaks()
+    out = {"peak_bf16_tflops": pk["bf16"], "layers": {}}
+    for l in layers:
+        c = l["case"]
+        t = make_layer_inputs(c)
+        w = L.svdq_prepare_weights(t.W_bits, t.act_absmax, t.bias_bits, rank=c.rank, fmt="int4")
+        xq, xsf, T = L.act_buffers(w, c.M, dev)
+
+        def layer():
+            L.svdq_quantize_act_lowrank_down(w, l["X"], xq, xsf, T)
+            L.svdq_linear_w4a4(w, xq, xsf, T, c.M, l["Y"])
+
+        def gemm():
+            L.svdq_linear_w4a4(w, xq, xsf, T, c.M, l["Y"])
+
+        us = 1e3 * _time_ms(torch, stream, layer, reps)
+        us_g = 1e3 * _time_ms(torch, stream, gemm, reps)
+        tf = c.flops / (us_g * 1e-6) / 1e12
+        out["layers"][c.name] = {"us": us, "gemm_us": us_g, "gemm_tflops": tf, "frac_of_bf16_peak": tf / pk["bf16"]}
+    return out
+
+
 def alpha_search(L, rows=256):
     """NEXT-3 (App. D migration strength): relative output error per candidate
     alpha on a calibration batch of one FLUX layer, through the library's own
@@ -407,7 +435,7 @@ def run_ours(args):
 
     # low-rank overhead: the same kernels at rank 0 (extras)
     overhead = None
-    unfused = sweep = small = refine = asearch = None
+    unfused = sweep = small = refine = asearch = int4 = None
     if args.extras:
         def step0():
             for l in layers:
@@ -432,6 +460,7 @@ def run_ours(args):
             small = small_m(L, torch, dev, stream)
             refine = refinement(L)
             asearch = alpha_search(L)
+            int4 = int4_layers(L, torch, layers, dev, stream)
 
     # end to end through the public host-buffer call: H2D of X, both kernels, D2H of Y
     e2e = None
@@ -488,6 +517,7 @@ def run_ours(args):
             "small_m_lora": small,
             "refinement": refine,
             "alpha_search": asearch,
+            "int4": int4,
             "gpu_launches": 2 * nl * args.steps,
             "e2e": e2e,
         }

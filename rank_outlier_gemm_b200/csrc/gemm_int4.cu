@@ -14,17 +14,19 @@
 // one step per 64-wide K group.
 //   warp 0      producer: per group, TMA of the packed codes (activations
 //               [128 x 32 B], weights [256 x 32 B]) and 1-D bulk copies of the
-//               group's bf16 scales into an 8-deep ring; per slab step, TMA of
-//               T and L2^T straight into a dequantized-tile buffer
+//               group's bf16 scales into a 6-deep ring; per slab step, TMA of
+//               T and L2^T into the slab buffer
 //   warp 1      MMA issuer: kind::f16 (fp16 operands for a group, bf16 for the
-//               slab), M128 N256 K16 x 4 per step, from the two dequantized-tile
-//               buffers
-//   warps 2-9   dequantizers: packed codes x scale -> fp16 tiles in the 128-byte
-//               swizzled K-major layout the MMA reads (a 16-byte chunk of 8
-//               values per thread and step), then an async-proxy fence
-//   warps 10-13 epilogue: tcgen05.ld, y = acc + b, bf16 RNE, 32-byte stores
+//               slab), M128 N256 K16 x 4 per group from the two dequantized-tile
+//               buffers, the slab from its own buffer
+//   warps 2-13  dequantizers: packed codes x scale -> fp16 tiles in the 128-byte
+//               swizzled K-major layout the MMA reads (one tile row of 64
+//               values per thread and group), then an async-proxy fence
+//   warps 14-17 epilogue: tcgen05.ld, y = acc + b, bf16 RNE, 32-byte stores
 // TMEM holds two 256-column accumulators, so one tile's epilogue overlaps the
-// next tile's main loop.  Launched as a programmatic dependent of the
+// next tile's main loop.  Each buffer has one writer and one reader that take
+// every one of its uses in turn (the slab has a buffer of its own): a parity
+// wait could not tell a phase from the one two uses earlier.  Launched as a programmatic dependent of the
 // activation kernel; the producer waits for it before its first load.
 #include <algorithm>
 #include <cstddef>
@@ -38,15 +40,16 @@ namespace {
 using namespace dev;
 
 constexpr int kBN = 256;
-constexpr int kThreads = 14 * 32;
-constexpr int kDqWarps = 8;
-constexpr int kPStages = 8;                        // packed-code ring
+constexpr int kThreads = 18 * 32;
+constexpr int kDqWarps = 12;                       // one tile row (128 + 256) per thread
+constexpr int kPStages = 6;                        // packed-code ring
 constexpr int kPA = 128 * 32;                      // activation codes of one group (128 rows)
 constexpr int kPB = kBN * 32;                      // weight codes of one group (256 rows)
 constexpr int kPStage = 13 * 1024;                 // codes + 256 + 512 bytes of scales, padded
 constexpr int kDA = 128 * 128;                     // dequantized activation tile: 128 rows x 64 fp16
 constexpr int kDB = kBN * 128;                     // dequantized weight tile: 256 rows x 64 fp16
 constexpr int kDBuf = kDA + kDB;
+constexpr int kSlab = 128 * 128 + kBN * 64;          // T (128 x 64 bf16) and L2^T (256 x 32 bf16)
 static_assert(kPA + kPB + 256 + 512 <= kPStage, "packed stage");
 
 struct K2IParams {
@@ -68,7 +71,8 @@ struct K2IShared {
   alignas(16) float bias[4][kBN];
   uint64_t pfull[kPStages];
   uint64_t pempty[kPStages];
-  uint64_t sfull[2];     // slab step landed in dequantized-tile buffer b (TMA)
+  uint64_t slab_full;    // a slab step landed in the slab buffer (TMA)
+  uint64_t slab_empty;   // the MMAs reading it have completed
   uint64_t dfull[2];     // dequantizers filled buffer b
   uint64_t dempty[2];    // the MMAs reading buffer b have completed
   uint64_t acc_full[2];
@@ -158,7 +162,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_int4_kernel(
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* dq = smem;                                  // 2 dequantized-tile buffers
-  uint8_t* pk = smem + 2 * kDBuf;                      // packed ring
+  uint8_t* sl = smem + 2 * kDBuf;                      // slab buffer
+  uint8_t* pk = sl + kSlab;                            // packed ring
   K2IShared* sh = reinterpret_cast<K2IShared*>(pk + kPStages * kPStage);
 
   const uint32_t warp = warp_id(), lane = lane_id();
@@ -170,8 +175,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_int4_kernel(
       mbar_init(&sh->pfull[s], 1);
       mbar_init(&sh->pempty[s], kDqWarps);
     }
+    mbar_init(&sh->slab_full, 1);
+    mbar_init(&sh->slab_empty, 1);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&sh->sfull[b], 1);
       mbar_init(&sh->dfull[b], kDqWarps);
       mbar_init(&sh->dempty[b], 1);
       mbar_init(&sh->acc_full[b], 1);
@@ -201,24 +207,21 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_int4_kernel(
         tma_prefetch_desc(&map_l2);
       }
       grid_dep_wait();  // the activation codes, scales and T come from the kernel ahead
-      int pst = 0, dst = 0;
-      int ns0 = 0, ns1 = 0;  // slab loads issued into buffer 0 / 1 (phases of sfull[b])
+      int pst = 0, sst = 0;  // packed stages and slab steps issued
       bool ok = true;
       for (int t = blockIdx.x; ok && t < ntiles_total; t += gridDim.x) {
         const int m0 = (t % p.mtiles) * 128;
         const int n0 = (t / p.mtiles) * kBN;
-        for (int k = 0; k < per_tile; ++k, ++dst) {
+        for (int k = 0; k < per_tile; ++k) {
           if (k < p.slab) {
-            const int b = dst & 1;
-            if (!wait_bounded(&sh->dempty[b], ((dst >> 1) & 1) ^ 1, wc)) {
+            if (!wait_bounded(&sh->slab_empty, (sst & 1) ^ 1, wc)) {
               ok = false;
               break;
             }
-            uint8_t* buf = dq + b * kDBuf;
-            mbar_arrive_expect_tx(&sh->sfull[b], kDA + kBN * 64);
-            tma_load_2d(buf, &map_t, &sh->sfull[b], 64 * k, m0);
-            tma_load_2d(buf + kDA, &map_l2, &sh->sfull[b], 32 * k, n0);
-            if (b) ++ns1; else ++ns0;
+            mbar_arrive_expect_tx(&sh->slab_full, kSlab);
+            tma_load_2d(sl, &map_t, &sh->slab_full, 64 * k, m0);
+            tma_load_2d(sl + 128 * 128, &map_l2, &sh->slab_full, 32 * k, n0);
+            ++sst;
           } else {
             const int g = k - p.slab;
             const int s = pst % kPStages;
@@ -239,8 +242,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_int4_kernel(
       if (sh->abort) {  // let copies in flight land before the CTA exits
         for (int i = max(0, pst - kPStages); i < pst; ++i)
           wait_drain(&sh->pfull[i % kPStages], (i / kPStages) & 1, p.wait_ns);
-        if (ns0 > 0) wait_drain(&sh->sfull[0], (ns0 - 1) & 1, p.wait_ns);
-        if (ns1 > 0) wait_drain(&sh->sfull[1], (ns1 - 1) & 1, p.wait_ns);
+        if (sst > 0) wait_drain(&sh->slab_full, (sst - 1) & 1, p.wait_ns);
       }
     }
   } else if (warp == 1) {
@@ -248,9 +250,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_int4_kernel(
     if (lane == 0) {
       const uint32_t id_f16 = idesc_f16(128, kBN);
       const uint32_t id_bf16 = idesc_bf16(128, kBN);
-      const uint32_t dq0 = smem_u32(dq);
-      int dst = 0, j = 0;
-      uint32_t ns = 0, nd = 0;  // completions of sfull[b] / dfull[b] consumed: bit b of the counts' parities
+      const uint32_t dq0 = smem_u32(dq), sl0 = smem_u32(sl);
+      int gst = 0, sst = 0, j = 0;  // group steps, slab steps, tiles
       bool ok = true;
       for (int t = blockIdx.x; ok && t < ntiles_total; t += gridDim.x, ++j) {
         const int a = j & 1;
@@ -258,18 +259,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_int4_kernel(
         tc_fence_after();
         const uint32_t acc = tmem + a * 256;
         uint32_t accum = 0;
-        for (int k = 0; k < per_tile; ++k, ++dst) {
-          const int b = dst & 1;
-          const uint32_t base = dq0 + b * kDBuf;
+        for (int k = 0; k < per_tile; ++k) {
           if (k < p.slab) {
-            const uint32_t ph = (ns >> b) & 1;
-            ns ^= 1u << b;
-            if (!wait_bounded(&sh->sfull[b], ph, wc)) {
+            if (!wait_bounded(&sh->slab_full, sst & 1, wc)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            const uint64_t da = desc_kmajor_sw128(base), dl = desc_kmajor_sw64(base + kDA);
+            const uint64_t da = desc_kmajor_sw128(sl0), dl = desc_kmajor_sw64(sl0 + 128 * 128);
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
               if (32 * k + 16 * c >= p.r_pad) break;
@@ -277,18 +274,21 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_int4_kernel(
               mma_bf16(acc, da + 4 * c + 2, dl + 2 * c, id_bf16, 1);      // T_lo
               accum = 1;
             }
+            mma_commit(&sh->slab_empty);
+            ++sst;
           } else {
-            const uint32_t ph = (nd >> b) & 1;
-            nd ^= 1u << b;
-            if (!wait_bounded(&sh->dfull[b], ph, wc)) {
+            const int b = gst & 1;
+            if (!wait_bounded(&sh->dfull[b], (gst >> 1) & 1, wc)) {
               ok = false;
               break;
             }
             tc_fence_after();
+            const uint32_t base = dq0 + b * kDBuf;
             mma_bf16_x4(acc, desc_kmajor_sw128(base), desc_kmajor_sw128(base + kDA), id_f16, accum);
             accum = 1;
+            mma_commit(&sh->dempty[b]);
+            ++gst;
           }
-          mma_commit(&sh->dempty[b]);
         }
         if (ok) mma_commit(&sh->acc_full[a]);
       }
@@ -296,40 +296,37 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_int4_kernel(
     }
   } else if (warp < 2 + kDqWarps) {
     // --------------------------------------------------------- dequantizers
-    const int tid = static_cast<int>(threadIdx.x) - 64;  // 0..255
-    int pst = 0, dst = 0;
+    // thread -> one row: activation rows 0..127, then weight rows 0..255
+    const int tid = static_cast<int>(threadIdx.x) - 64;  // 0..383
+    const bool is_a = tid < 128;
+    const int row = is_a ? tid : tid - 128;
+    const int code_off = (is_a ? 0 : kPA) + row * 32;
+    const int out_off = (is_a ? 0 : kDA) + (row >> 3) * 1024 + (row & 7) * 128;
+    int pst = 0;  // group steps (packed stages = uses of the dequantized-tile buffers)
     bool ok = true;
     for (int t = blockIdx.x; ok && t < ntiles_total; t += gridDim.x) {
-      for (int k = 0; k < per_tile; ++k, ++dst) {
-        if (k < p.slab) continue;  // the producer fills this buffer with T and L2 directly
+      for (int g = 0; g < p.groups; ++g) {
         const int s = pst % kPStages;
-        const int b = dst & 1;
+        const int b = pst & 1;
         if (!wait_warp(&sh->pfull[s], (pst / kPStages) & 1, wc)) {
           ok = false;
           break;
         }
-        if (!wait_warp(&sh->dempty[b], ((dst >> 1) & 1) ^ 1, wc)) {
+        if (!wait_warp(&sh->dempty[b], ((pst >> 1) & 1) ^ 1, wc)) {
           ok = false;
           break;
         }
         const uint8_t* st = pk + s * kPStage;
-        const uint16_t* sa = reinterpret_cast<const uint16_t*>(st + kPA + kPB);
-        const uint16_t* sb = sa + 128;
-        uint8_t* out = dq + b * kDBuf;
-        // 16-byte chunk i: rows 0..127 of the activation tile, then 256 weight rows
-#pragma unroll 4
-        for (int i = tid; i < (128 + kBN) * 8; i += 256) {
-          const bool is_a = i < 128 * 8;
-          const int ii = is_a ? i : i - 128 * 8;
-          const int row = ii >> 3, c = ii & 7;
-          const uint32_t w = *reinterpret_cast<const uint32_t*>(st + (is_a ? 0 : kPA) + row * 32 + c * 4);
-          const float sf = __uint_as_float(static_cast<uint32_t>(is_a ? sa[row] : sb[row]) << 16);
-          const __half sh16 = __float2half_rn(sf);
-          const uint4 v = int4x8_to_f16x8(w, __halves2half2(sh16, sh16));
-          // 128-byte swizzle: chunk c of row r at chunk c ^ (r % 8), 8-row groups of 1024 bytes
-          *reinterpret_cast<uint4*>(out + (is_a ? 0 : kDA) + (row >> 3) * 1024 + (row & 7) * 128 +
-                                    ((c ^ (row & 7)) << 4)) = v;
-        }
+        const uint16_t* scales = reinterpret_cast<const uint16_t*>(st + kPA + kPB);  // 128 then 256
+        const uint4 c0 = *reinterpret_cast<const uint4*>(st + code_off);
+        const uint4 c1 = *reinterpret_cast<const uint4*>(st + code_off + 16);
+        const __half sh16 = __float2half_rn(__uint_as_float(static_cast<uint32_t>(scales[tid]) << 16));
+        const __half2 s2 = __halves2half2(sh16, sh16);
+        const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};  // 8 codes each
+        uint8_t* orow = dq + b * kDBuf + out_off;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)  // 128-byte swizzle: chunk c of row r at chunk c ^ (r % 8)
+          *reinterpret_cast<uint4*>(orow + ((c ^ (row & 7)) << 4)) = int4x8_to_f16x8(cw[c], s2);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the tensor core
         __syncwarp();
         if (lane == 0) {
@@ -427,7 +424,7 @@ svdq_status launch_gemm_int4(const GemmInt4Args& a, cudaStream_t stream) {
   }
   const CUtensorMap& map_l2 = a.r_pad > 0 ? *a.map_l2_256 : map_xq;
 
-  const size_t smem = 1024 + 2 * static_cast<size_t>(kDBuf) + static_cast<size_t>(kPStages) * kPStage +
+  const size_t smem = 1024 + 2 * static_cast<size_t>(kDBuf) + kSlab + static_cast<size_t>(kPStages) * kPStage +
                       sizeof(K2IShared);
   static bool attr_set[64] = {};
   int cur_dev = 0;

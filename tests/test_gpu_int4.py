@@ -165,3 +165,21 @@ def test_int4_library_prepare():
     assert e4 < 0.1 and ef < 0.1, (e4, ef)
     with pytest.raises(Exception):
         L.svdq_prepare_weights(t.W_bits, t.act_absmax, t.bias_bits, rank=32, fmt="int4", refine_iters=2)
+
+
+def test_int4_full_size_layer_repeatable():
+    """FLUX attn_out at full size (36 x 12 tiles, several per CTA, so every
+    buffer of the GEMM's rings turns over many times): rows from the start,
+    middle and end within the layer tolerance of the oracle, and two launches
+    bitwise equal."""
+    L = G.lib()
+    case, t, prep = _case("flux/attn_out", 4608)
+    w = _weights(prep)
+    Y, (xq, xsf, T) = G.run_layer(w, t.X_bits)
+    rows = np.r_[0:40, 2300:2340, case.M - 40:case.M]
+    G.check_Y(Y[rows], OI.linear(prep, t.X, rows=rows))
+    Y2 = torch.empty((case.M, case.N), dtype=torch.bfloat16, device="cuda")
+    for _ in range(3):
+        L.svdq_linear_w4a4(w, xq, xsf, T, case.M, Y2)
+    assert L.svdq_check_device_errors() == 0
+    np.testing.assert_array_equal(Y2.float().cpu().numpy(), Y)
