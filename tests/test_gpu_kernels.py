@@ -384,3 +384,24 @@ def test_bounded_wait_reports_timeout():
     # the context is still usable and the error word was cleared
     Y, _ = G.run_layer(w, t.X_bits)
     G.check_Y(Y, OS.linear(prep, t.X))
+
+
+def test_full_size_layer_repeatable():
+    """FLUX attn_out at full size (36 x 12 tiles over 148 persistent CTAs, so
+    each CTA hands its accumulators and scale slots over between tiles): rows
+    from the start, middle and end within the layer tolerance of the oracle,
+    codes and scales of those rows bit-exact, and repeated launches bitwise
+    equal."""
+    L = G.lib()
+    t, prep = _case_prep("flux/attn_out", 4608)
+    w = G.weights_from_oracle(prep)
+    Y, (xq, xsf, T) = G.run_layer(w, t.X_bits)
+    M, N = Y.shape
+    rows = np.r_[0:40, 2300:2340, M - 40:M]
+    G.check_codes(xq, xsf, t.X, prep.inv_lam, rows=rows)
+    G.check_Y(Y[rows], OS.linear(prep, t.X, rows=rows))
+    Y2 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    for _ in range(3):
+        L.svdq_linear_w4a4(w, xq, xsf, T, M, Y2)
+    assert L.svdq_check_device_errors() == 0
+    np.testing.assert_array_equal(Y2.float().cpu().numpy(), Y)
