@@ -359,8 +359,9 @@ def run_ours(args):
     layers = []
     for c in cases:
         t = make_layer_inputs(c)
-        w = L.svdq_prepare_weights(t.W_bits, t.act_absmax, t.bias_bits, rank=c.rank)
-        w0 = L.svdq_prepare_weights(t.W_bits, t.act_absmax, t.bias_bits, rank=0) if args.extras else None
+        w = L.svdq_prepare_weights(t.W_bits, t.act_absmax, t.bias_bits, rank=c.rank, fmt=args.format)
+        w0 = (L.svdq_prepare_weights(t.W_bits, t.act_absmax, t.bias_bits, rank=0, fmt=args.format)
+              if args.extras else None)
         X = torch.from_numpy(t.X_bits.view(np.int16).copy()).view(torch.bfloat16).to(dev)
         bufs = L.act_buffers(w, c.M, dev)
         Y = torch.empty((c.M, c.N), dtype=torch.bfloat16, device=dev)
@@ -423,10 +424,15 @@ def run_ours(args):
     capped = bool(cl) and ("sw_power_cap" in cl["reasons"] or
                            (cl["sm_mhz"] or 0) < 0.95 * (cl["sm_max_mhz"] or 1))
     bf16_peak = pk["bf16_sustained"] if capped else pk["bf16"]
-    fp4_peak = bf16_peak * NOMINAL_FP4_OVER_BF16
-    peak_src = (f"{pk['source']} bf16 {'sustained' if capped else 'burst'} {bf16_peak} x "
-                f"{NOMINAL_FP4_OVER_BF16} (nominal FP4:BF16)")
-    traffic, traffic_note = k2_traffic_per_launch([l["case"].name for l in layers])
+    if args.format == "int4":  # the INT4 GEMM contracts fp16 tiles dequantized on chip
+        fp4_peak = bf16_peak
+        peak_src = f"{pk['source']} bf16 {'sustained' if capped else 'burst'} {bf16_peak} (fp16 contraction)"
+        traffic, traffic_note = None, "no ncu counters kept for the INT4 GEMM in bench.py"
+    else:
+        fp4_peak = bf16_peak * NOMINAL_FP4_OVER_BF16
+        peak_src = (f"{pk['source']} bf16 {'sustained' if capped else 'burst'} {bf16_peak} x "
+                    f"{NOMINAL_FP4_OVER_BF16} (nominal FP4:BF16)")
+        traffic, traffic_note = k2_traffic_per_launch([l["case"].name for l in layers])
     k2_flops = flops_step
     k2_ms = sum(k2)
     achieved = k2_flops / (k2_ms * 1e-3) / 1e12
@@ -460,7 +466,7 @@ def run_ours(args):
             small = small_m(L, torch, dev, stream)
             refine = refinement(L)
             asearch = alpha_search(L)
-            int4 = int4_layers(L, torch, layers, dev, stream)
+            int4 = int4_layers(L, torch, layers, dev, stream) if args.format == "nvfp4" else None
 
     # end to end through the public host-buffer call: H2D of X, both kernels, D2H of Y
     e2e = None
@@ -495,8 +501,9 @@ def run_ours(args):
         out = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic (seeded; FLUX.1 shapes, random weights)",
-            "config": {"workload": WORKLOAD, "M": cases[0].M, "layers": [[c.K, c.N] for c in cases],
+            "vs_baseline": None, "dtype": args.format, "data": "synthetic (seeded; FLUX.1 shapes, random weights)",
+            "config": {"workload": WORKLOAD, "format": args.format, "M": cases[0].M,
+                       "layers": [[c.K, c.N] for c in cases],
                        "rank": cases[0].rank, "parallelism": f"replicas x{world}",
                        "l2": "step footprint ~0.5 GB > 126 MB L2; no flush"},
             "breakdown_note": ("us_per_layer / us_act_kernel / us_gemm_kernel come from a second pass of the "
@@ -509,7 +516,8 @@ def run_ours(args):
             "frac_of_layer_roofline": sum(roof_us.values()) / (1e3 * (sum(k1) + sum(k2))),
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
                          "frac": achieved / fp4_peak, "traffic": traffic, "traffic_note": traffic_note,
-                         "kernel": "gemm_w4a4_kernel", "peak_source": peak_src,
+                         "kernel": "gemm_int4_kernel" if args.format == "int4" else "gemm_w4a4_kernel",
+                         "peak_source": peak_src,
                          "frac_of_datasheet_9pf": achieved / 9000.0},
             "lowrank_overhead_vs_rank0": overhead,
             "unfused_lowrank_overhead_vs_rank0": unfused,
@@ -619,6 +627,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--no-extras", dest="extras", action="store_false")
     ap.add_argument("--layers", default="", help="comma-separated subset of the FLUX layers (profiling)")
+    ap.add_argument("--format", choices=["nvfp4", "int4"], default="nvfp4",
+                    help="4-bit format of the timed step (INT4: the variant with group-64 bf16 scales)")
     args = ap.parse_args()
     global LAYER_FILTER
     LAYER_FILTER = [x for x in args.layers.split(",") if x] or None
