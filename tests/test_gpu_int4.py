@@ -183,3 +183,53 @@ def test_int4_full_size_layer_repeatable():
         L.svdq_linear_w4a4(w, xq, xsf, T, case.M, Y2)
     assert L.svdq_check_device_errors() == 0
     np.testing.assert_array_equal(Y2.float().cpu().numpy(), Y)
+
+
+def test_int4_cuda_graph_capture_and_replay():
+    """The INT4 forward pass (activation kernel, then the GEMM as its
+    programmatic dependent) captured into a CUDA graph replays to the eager
+    output and follows a rewrite of the captured input."""
+    L = G.lib()
+    case, t, prep = _case("pixart/mlp_up", 300)
+    w = _weights(prep)
+    M, N = t.X_bits.shape[0], w.info["N"]
+    X = G.to_dev_bf16(t.X_bits)
+    X2 = G.to_dev_bf16(t.X_bits[::-1].copy())
+    ws = torch.empty(L.svdq_forward_workspace_bytes(w, M), dtype=torch.uint8, device="cuda")
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    eager = []
+    for src in (X, X2):
+        L.svdq_forward(w, src, Y, ws)
+        eager.append(Y.clone())
+    torch.cuda.synchronize()
+    Xg = X.clone()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        L.svdq_forward(w, Xg, Y, ws)
+    Y.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(Y, eager[0])
+    Xg.copy_(X2)
+    g.replay()
+    torch.cuda.synchronize()
+    assert L.svdq_check_device_errors() == 0
+    assert torch.equal(Y, eager[1])
+    del g
+
+
+def test_int4_alpha_search_runs_on_the_int4_layer():
+    """svdq_search_alpha with the INT4 format scores every candidate through the
+    INT4 kernels; its errors are finite, the pick is the smallest, and the
+    α = 0.5 score matches preparing at 0.5 and measuring the output directly."""
+    L = G.lib()
+    case, t, _ = _case("tiny/layer", 64)
+    alphas = (0.3, 0.5, 0.7)
+    errs, best = L.svdq_search_alpha(t.W_bits, t.X_bits, t.bias_bits, alphas=alphas, rank=case.rank, fmt="int4")
+    assert len(errs) == 3 and all(np.isfinite(errs)) and best == int(np.argmin(errs))
+    w = L.svdq_prepare_weights(t.W_bits, np.abs(t.X).max(axis=0), t.bias_bits, rank=case.rank, alpha=0.5,
+                               fmt="int4")
+    Y, _ = G.run_layer(w, t.X_bits)
+    exact = t.X.astype(np.float64) @ t.W.astype(np.float64).T + t.bias
+    # the library scores against an fp32 reference; the float64 one differs in the last bits
+    assert abs(errs[1] - np.linalg.norm(Y - exact) / np.linalg.norm(exact)) < 1e-4
