@@ -206,7 +206,8 @@ svdq_status svdq_quantize_act_lowrank_down(const svdq_weights* w, const void* X_
 
 /*
  * For an INT4 handle the same call writes INT4 codes (two's-complement
- * nibbles, element 2i in the low half of byte i) into xq and bf16 scales,
+ * nibbles; per 8 elements one little-endian 32-bit word holding elements
+ * 0, 2, 4, 6 in nibbles 0-3 and 1, 3, 5, 7 in nibbles 4-7) into xq and bf16 scales,
  * group-major [K/64][round_up(M, 128)] with zeros for the padding rows, into
  * xsf; the buffer sizes above cover both formats.
  */

@@ -24,8 +24,11 @@ the layer has no per-tensor weight factor (bf16 scales span fp32's exponent
 range).  Everything else -- smoothing, the low-rank split, the residual, LoRA
 -- is the NVFP4 layer's (``svdquant.py``).
 
-Storage: codes are two's-complement nibbles, two per byte, element 2i in the
-low nibble; scales are bf16 bit patterns, stored group-major ([K/64, rows]).
+Storage (not fixed by the pages; chosen so that the GEMM unpacks pairs of
+consecutive elements without byte permutes): codes are two's-complement
+nibbles; each run of 8 elements is a little-endian 32-bit word whose nibbles
+0-3 hold the even elements (0, 2, 4, 6) and nibbles 4-7 the odd ones
+(1, 3, 5, 7).  Scales are bf16 bit patterns, stored group-major ([K/64, rows]).
 """
 
 from __future__ import annotations
@@ -72,18 +75,28 @@ def dequantize_groups(codes, scales) -> np.ndarray:
 
 
 def pack_codes(codes) -> np.ndarray:
-    """Two's-complement nibbles, two per byte, element 2i low: uint8 [R, K/2]."""
+    """uint8 [R, K/2]: per 8 elements a little-endian word with the even
+    elements in nibbles 0-3 and the odd ones in nibbles 4-7."""
     c = np.asarray(codes, np.int64) & 0xF
-    return (c[:, 0::2] | (c[:, 1::2] << 4)).astype(np.uint8)
+    R, K = c.shape
+    c = c.reshape(R, K // 8, 8)
+    word = np.zeros((R, K // 8), np.uint64)
+    for k in range(4):
+        word |= (c[..., 2 * k].astype(np.uint64) << np.uint64(4 * k)) | \
+                (c[..., 2 * k + 1].astype(np.uint64) << np.uint64(16 + 4 * k))
+    return word.astype("<u4").view(np.uint8).reshape(R, K // 2)
 
 
 def unpack_codes(packed) -> np.ndarray:
     """Inverse of pack_codes: int8 [R, K]."""
-    p = np.asarray(packed, np.int64)
-    lo, hi = p & 0xF, (p >> 4) & 0xF
-    out = np.empty((p.shape[0], 2 * p.shape[1]), np.int64)
-    out[:, 0::2] = lo
-    out[:, 1::2] = hi
+    p = np.ascontiguousarray(np.asarray(packed, np.uint8))
+    R = p.shape[0]
+    word = p.view("<u4").astype(np.int64)
+    out = np.empty((R, word.shape[1], 8), np.int64)
+    for k in range(4):
+        out[..., 2 * k] = (word >> (4 * k)) & 0xF
+        out[..., 2 * k + 1] = (word >> (16 + 4 * k)) & 0xF
+    out = out.reshape(R, -1)
     return np.where(out >= 8, out - 16, out).astype(np.int8)
 
 

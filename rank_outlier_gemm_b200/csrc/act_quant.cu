@@ -20,7 +20,8 @@
 // The INT4 instantiation (SVDQuant App. D: groups of 64, 16-bit scales; §3:
 // qmax 7) quantizes each row's 64-column tile as one group: the lane pair
 // holding its two halves combines their maxima, s = bf16(fp32(amax / 7)),
-// q = clamp(rint(fp32(v * fp32(1 / s))), -7, 7), two's-complement nibbles,
+// q = clamp(rint(fp32(v * fp32(1 / s))), -7, 7), two's-complement nibbles (per
+// 8 elements one word, even elements in nibbles 0-3, odd ones in 4-7),
 // and the bf16 scale goes to a group-major [K/64][rows padded to 128] array.
 #include <cooperative_groups.h>
 
@@ -80,13 +81,14 @@ __device__ __forceinline__ void bar_sync_quant() {
   asm volatile("bar.sync 1, %0;" ::"n"(kQuantWarps * 32) : "memory");
 }
 
-// INT4: eight codes (element i in bits 4i..4i+3) of v[0..7] times r.
+// INT4: the eight codes of v[0..7] times r as one word, even elements in
+// nibbles 0-3 and odd ones in nibbles 4-7.
 __device__ __forceinline__ uint32_t int4x8(const float* v, float r) {
   uint32_t w = 0;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int q = min(7, max(-7, __float2int_rn(__fmul_rn(v[i], r))));
-    w |= (static_cast<uint32_t>(q) & 0xFu) << (4 * i);
+    w |= (static_cast<uint32_t>(q) & 0xFu) << (4 * ((i & 1) ? 4 + (i >> 1) : (i >> 1)));
   }
   return w;
 }

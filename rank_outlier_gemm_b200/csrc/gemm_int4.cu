@@ -90,23 +90,15 @@ __device__ __noinline__ bool wait_drain(uint64_t* bar, uint32_t parity, uint64_t
   return true;
 }
 
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
-  uint32_t r;
-  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
-  return r;
-}
-
-// Eight two's-complement INT4 codes (element i in bits 4i..4i+3) times scale s
-// -> eight fp16 values in element order.  Offset-binary nibbles OR'ed into the
-// fp16 pattern of 1024 give 1024 + (q + 8) exactly; subtracting 1032 gives q.
+// Eight two's-complement INT4 codes (elements 2k in nibble k, 2k+1 in nibble
+// k + 4) times scale s -> eight fp16 values in element order.  Offset-binary
+// nibbles OR'ed into the fp16 pattern of 1024 give 1024 + (q + 8) exactly;
+// subtracting 1032 gives q.  Mask k picks nibbles k and k + 4, i.e. elements
+// 2k and 2k + 1, already in the low and high halves of a half2.
 __device__ __forceinline__ uint4 int4x8_to_f16x8(uint32_t w, __half2 s2) {
   const uint32_t u = w ^ 0x88888888u;
-  const uint32_t p04 = (u & 0x000F000Fu) | 0x64006400u;          // elements 0 and 4
-  const uint32_t p15 = ((u >> 4) & 0x000F000Fu) | 0x64006400u;   // 1 and 5
-  const uint32_t p26 = ((u >> 8) & 0x000F000Fu) | 0x64006400u;   // 2 and 6
-  const uint32_t p37 = ((u >> 12) & 0x000F000Fu) | 0x64006400u;  // 3 and 7
-  const uint32_t in[4] = {prmt(p04, p15, 0x5410u), prmt(p26, p37, 0x5410u),
-                          prmt(p04, p15, 0x7632u), prmt(p26, p37, 0x7632u)};
+  const uint32_t in[4] = {(u & 0x000F000Fu) | 0x64006400u, ((u >> 4) & 0x000F000Fu) | 0x64006400u,
+                          ((u >> 8) & 0x000F000Fu) | 0x64006400u, ((u >> 12) & 0x000F000Fu) | 0x64006400u};
   const __half2 bias = __halves2half2(__ushort_as_half(0x6408u), __ushort_as_half(0x6408u));  // 1032
   uint32_t out[4];
 #pragma unroll

@@ -377,14 +377,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
       for (int k = 0; k < per_tile; ++k, ++it) {
         const int s = it % kStages;
         const uint32_t ph = (it / kStages) & 1;
-        if (k == nslab) {
-          // the scale buffers live in acc[a^1]: wait until the previous tile's
-          // epilogue has read its first 96 columns
-          if (!wait_warp(&sh->sfreg_free[a ^ 1], ((j - 1) >> 1) & 1, wc)) {
-            ok = false;
-            break;
-          }
-        }
         if (k >= nslab) {
           if (!wait_warp(&sh->full[s], ph, wc)) {
             ok = false;
@@ -413,6 +405,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(&sh->empty[s]);
+          if (k == nslab) {
+            // the scale slots live in acc[a^1]: before the tile's first store into
+            // them, wait until the previous tile's epilogue has read its first 96 columns
+            if (!wait_warp(&sh->sfreg_free[a ^ 1], ((j - 1) >> 1) & 1, wc)) {
+              ok = false;
+              break;
+            }
+          }
           const int b = sfi & (kSfSlots - 1);
           if (!wait_warp(&sh->sf_empty[b], ((sfi / kSfSlots) & 1) ^ 1, wc)) {
             ok = false;

@@ -57,8 +57,9 @@ float weight_factor(const float* R, size_t n) {
 
 // INT4 codec (SVDQuant App. D: groups of 64 with 16-bit scales; §3: qmax 7):
 // s = bf16(fp32(amax / 7)), q = clamp(rint(fp32(v * fp32(1 / s))), -7, 7) with
-// round-half-even, two's-complement nibbles with element 2i in the low half
-// of byte i.  IEEE fp32 host arithmetic (no contraction across the steps).
+// round-half-even, two's-complement nibbles, per 8 elements one little-endian
+// word with the even elements in nibbles 0-3 and the odd ones in nibbles 4-7.
+// IEEE fp32 host arithmetic (no contraction across the steps).
 void int4_encode_rows(const float* R, int rows, int K, int rows_pad, uint8_t* codes, uint16_t* scales) {
   const int G = K / 64;
   for (int n = 0; n < rows; ++n) {
@@ -72,13 +73,14 @@ void int4_encode_rows(const float* R, int rows, int K, int rows_pad, uint8_t* co
       scales[static_cast<size_t>(g) * rows_pad + n] = sb;
       const float sv = bf16_to_f32(sb);
       volatile float r = sv > 0.0f ? 1.0f / sv : 0.0f;
-      for (int j = 0; j < 64; j += 2) {
-        int q[2];
-        for (int e = 0; e < 2; ++e) {
+      for (int j = 0; j < 64; j += 8) {
+        uint32_t word = 0;
+        for (int e = 0; e < 8; ++e) {
           volatile float t = v[64 * g + j + e] * r;
-          q[e] = std::min(7, std::max(-7, static_cast<int>(std::nearbyint(t))));
+          const int q = std::min(7, std::max(-7, static_cast<int>(std::nearbyint(t))));
+          word |= (static_cast<uint32_t>(q) & 0xFu) << (4 * ((e & 1) ? 4 + (e >> 1) : (e >> 1)));
         }
-        c[32 * g + j / 2] = static_cast<uint8_t>((q[0] & 0xF) | ((q[1] & 0xF) << 4));
+        for (int b = 0; b < 4; ++b) c[32 * g + j / 2 + b] = static_cast<uint8_t>(word >> (8 * b));
       }
     }
   }

@@ -90,7 +90,9 @@ def test_pack_unpack():
     p = OI.pack_codes(q)
     assert p.shape == (5, 64) and p.dtype == np.uint8
     np.testing.assert_array_equal(OI.unpack_codes(p), q)
-    np.testing.assert_array_equal(OI.pack_codes(np.array([[1, -1, -7, 7]], np.int8)), [[0xF1, 0x79]])
+    # nibbles (two's complement) 1, F, 9, 7, 0, 2, 3, D; evens 1 9 0 3 -> 0x3091, odds F 7 2 D -> 0xD27F
+    np.testing.assert_array_equal(OI.pack_codes(np.array([[1, -1, -7, 7, 0, 2, 3, -3]], np.int8)),
+                                  [[0x91, 0x30, 0x7F, 0xD2]])
 
 
 def test_scale_bits_roundtrip():
