@@ -61,10 +61,10 @@ def peaks():
 # kernel source the counters were taken on; counters of another source are stale
 # and not reported.
 K2_TRAFFIC = {
-    "source_sha256": "fd419957ddb1a472fbbb8a953913cd3986f4fcd27e446f5a569aad328deeacb0",
+    "source_sha256": "11554d84cb53683ba96d19403a047117614bfa2844fec6ffc17f189da222e94f",
     # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum: read + write per launch
-    "bytes_per_launch": {"attn_out": 14118656 + 1536, "qkv": 25145088 + 31958272,
-                         "mlp_up": 30719744 + 59113472, "mlp_down": 56924928 + 6905856},
+    "bytes_per_launch": {"attn_out": 14110464 + 1792, "qkv": 25147648 + 32385280,
+                         "mlp_up": 30663680 + 59214336, "mlp_down": 56352512 + 6549248},
 }
 
 
