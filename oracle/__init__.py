@@ -11,9 +11,10 @@ Modules:
   codec     NVFP4 group-16 codec, nibble packing, block-scale atom layout
   svdquant  smoothing, SVD split, residual, weight factor, output, LoRA
   int4      INT4 variant: group-64 codec with bf16 scales, nibble packing, output
+  norm      LayerNorm + per-channel modulation in front of the layer (fused path)
 
 Parity status: every function is pinned by a CPU test against library casts,
 brute force, closed forms or invariants (tests/test_oracle_*.py).
 """
 
-from . import codec, formats, int4, svdquant  # noqa: F401
+from . import codec, formats, int4, norm, svdquant  # noqa: F401
