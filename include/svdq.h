@@ -234,6 +234,41 @@ svdq_status svdq_linear_w4a4(const svdq_weights* w, const void* xq, const void* 
                              const void* T, int M, void* Y_bf16, void* stream);
 
 /*
+ * The activation kernel fused with the adaLN front end of a DiT block
+ * (SVDQuant §4.3 fuses the down-projection into the quantization kernel; this
+ * extends the fusion to the norm ahead of the layer): per token
+ * x_j = bf16(fp32(fp32(fp32(z_j - mu) * rstd) * a_j) + c_j), then exactly what
+ * svdq_quantize_act_lowrank_down does with X = x.  The pre-norm activations are
+ * read in place of X (the layer never stores X).
+ *   Z_bf16   device, M x K bf16 pre-norm activations
+ *   stats    device, M x 2 floats (mu, rstd) from svdq_act_row_stats
+ *   norm_a   device, K floats (1 + scale);  norm_c  device, K floats (shift)
+ *   xq, xsf, T as for svdq_quantize_act_lowrank_down
+ */
+svdq_status svdq_norm_quantize_act_lowrank_down(const svdq_weights* w, const void* Z_bf16, int M,
+                                                const float* stats, const float* norm_a,
+                                                const float* norm_c, void* xq, void* xsf, void* T,
+                                                void* stream);
+
+/*
+ * LayerNorm statistics per token: mu = mean_j z_j and
+ * rstd = 1 / sqrt(mean_j (z_j - mu)^2 + eps), accumulated in fp32 (two passes
+ * over the row), IEEE square root and reciprocal.
+ *   Z_bf16  device, M x K bf16;  stats  device, M x 2 floats (out)
+ * SVDQ_ERR_INVALID_ARG for bad sizes, eps < 0 or misaligned pointers.
+ */
+svdq_status svdq_act_row_stats(const void* Z_bf16, int M, int K, float eps, float* stats, void* stream);
+
+/*
+ * The layer with the norm in front: row statistics, the fused activation
+ * kernel and the GEMM.  `workspace` is device memory of at least
+ * svdq_forward_norm_workspace_bytes(w, M) bytes.
+ */
+svdq_status svdq_forward_norm(const svdq_weights* w, const void* Z_bf16, int M, const float* norm_a,
+                              const float* norm_c, float eps, void* Y_bf16, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
+/*
  * Both kernels back to back.  `workspace` is device memory of at least
  * svdq_forward_workspace_bytes(w, M) bytes holding xq, xsf and T.
  */
@@ -286,6 +321,7 @@ size_t svdq_act_sf_bytes(int M, int K);                    /* ceil(M/128)*128 * 
 size_t svdq_lowrank_bytes(const svdq_weights* w, int M);   /* M * 2 * r_pad * 2 */
 size_t svdq_forward_workspace_bytes(const svdq_weights* w, int M);
 size_t svdq_forward_host_workspace_bytes(const svdq_weights* w, int M);
+size_t svdq_forward_norm_workspace_bytes(const svdq_weights* w, int M);
 size_t svdq_weights_sf_bytes(const svdq_weights* w);       /* the handle's weight scales */
 
 /* Shape of a handle: rank counts the SVD rank plus attached LoRA ranks, r_pad

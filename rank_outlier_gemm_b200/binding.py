@@ -53,6 +53,10 @@ _SIGS = {
     "svdq_forward": (_i, [_vp, _vp, _i, _vp, _vp, _sz, _vp]),
     "svdq_forward_host": (_i, [_vp, _vp, _i, _vp, _vp, _sz, _vp]),
     "svdq_forward_noalloc": (_i, [_vp, _vp, _i, _vp, _vp]),
+    "svdq_act_row_stats": (_i, [_vp, _i, _i, _f, _vp, _vp]),
+    "svdq_norm_quantize_act_lowrank_down": (_i, [_vp, _vp, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "svdq_forward_norm": (_i, [_vp, _vp, _i, _vp, _vp, _f, _vp, _vp, _sz, _vp]),
+    "svdq_forward_norm_workspace_bytes": (_sz, [_vp, _i]),
     "svdq_act_codes_bytes": (_sz, [_i, _i]),
     "svdq_act_sf_bytes": (_sz, [_i, _i]),
     "svdq_lowrank_bytes": (_sz, [_vp, _i]),
@@ -239,6 +243,31 @@ def svdq_forward_noalloc(w: Weights, X: torch.Tensor, Y: torch.Tensor, stream=No
     """svdq_forward with the intermediates in the library's static device block (no allocation)."""
     _check(_lib.svdq_forward_noalloc(w.handle, _dev(X, "X"), X.shape[0], _dev(Y, "Y"), _stream(stream)),
            "svdq_forward_noalloc")
+
+
+def svdq_act_row_stats(Z: torch.Tensor, eps: float, stats: torch.Tensor, stream=None) -> None:
+    """(mu, rstd) per row of a CUDA bf16 [M, K] tensor into a CUDA float32 [M, 2] tensor."""
+    _check(_lib.svdq_act_row_stats(_dev(Z, "Z"), Z.shape[0], Z.shape[1], float(eps), _dev(stats, "stats"),
+                                   _stream(stream)), "svdq_act_row_stats")
+
+
+def svdq_norm_quantize_act_lowrank_down(w: Weights, Z: torch.Tensor, stats: torch.Tensor, norm_a: torch.Tensor,
+                                        norm_c: torch.Tensor, xq, xsf, T, stream=None) -> None:
+    _check(_lib.svdq_norm_quantize_act_lowrank_down(w.handle, _dev(Z, "Z"), Z.shape[0], _dev(stats, "stats"),
+                                                    _dev(norm_a, "norm_a"), _dev(norm_c, "norm_c"), _dev(xq, "xq"),
+                                                    _dev(xsf, "xsf"), _dev(T, "T"), _stream(stream)),
+           "svdq_norm_quantize_act_lowrank_down")
+
+
+def svdq_forward_norm(w: Weights, Z: torch.Tensor, norm_a: torch.Tensor, norm_c: torch.Tensor, eps: float,
+                      Y: torch.Tensor, workspace: torch.Tensor, stream=None) -> None:
+    _check(_lib.svdq_forward_norm(w.handle, _dev(Z, "Z"), Z.shape[0], _dev(norm_a, "norm_a"), _dev(norm_c, "norm_c"),
+                                  float(eps), _dev(Y, "Y"), _dev(workspace, "workspace"),
+                                  workspace.numel() * workspace.element_size(), _stream(stream)), "svdq_forward_norm")
+
+
+def svdq_forward_norm_workspace_bytes(w: Weights, M: int) -> int:
+    return _lib.svdq_forward_norm_workspace_bytes(w.handle, M)
 
 
 def svdq_act_codes_bytes(M: int, K: int) -> int:

@@ -23,6 +23,13 @@
 // q = clamp(rint(fp32(v * fp32(1 / s))), -7, 7), two's-complement nibbles (per
 // 8 elements one word, even elements in nibbles 0-3, odd ones in 4-7),
 // and the bf16 scale goes to a group-major [K/64][rows padded to 128] array.
+//
+// The norm instantiation reads the pre-norm activations Z instead of X and
+// first applies the adaLN front end of the configured DiT blocks per element,
+// x = bf16(((z - mu) * rstd) * a_j + c_j) with the row's mu and rstd from the
+// row-statistics kernel (zero for padding rows).  Each quantizer thread writes
+// its normalized values back into the stage's tile, so the down-projection MMA
+// (which waits for that) and the quantizer both see X; the rest is unchanged.
 #include <cooperative_groups.h>
 
 #include <algorithm>
@@ -54,6 +61,9 @@ struct K1Params {
   uint64_t wait_ns;
   int stall;
   int m_pad;           // INT4: rows of the group-major scale array
+  const float2* stats;  // norm: (mu, rstd) per row
+  const float* norm_a;  // norm: per-channel multiplier [K]
+  const float* norm_c;  // norm: per-channel offset [K]
   uint32_t l1_tile;    // r_pad * 128 bytes
   uint32_t tmem_cols;
 };
@@ -62,6 +72,7 @@ struct K1Shared {
   float rcp_tbl[16];  // reciprocals of the E4M3 mantissa patterns (see nvfp4.cuh)
   uint64_t full[kStages];
   uint64_t empty[kStages];
+  uint64_t normed[kStages];  // norm: the quantizer warps wrote X into the stage
   uint64_t tfull;
   uint64_t never;
   uint32_t tmem_base;
@@ -93,7 +104,7 @@ __device__ __forceinline__ uint32_t int4x8(const float* v, float r) {
   return w;
 }
 
-template <bool kInt4>
+template <bool kInt4, bool kNorm>
 __global__ void __launch_bounds__(kThreads, 2) act_quant_lowrank_kernel(
     const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_l1,
     const K1Params p) {
@@ -101,8 +112,9 @@ __global__ void __launch_bounds__(kThreads, 2) act_quant_lowrank_kernel(
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* xs = smem;
   uint8_t* l1s = xs + kStages * kXTile;
+  constexpr int kAux = kInvTile * (kNorm ? 3 : 1);  // inv_lam (then a and c) of a tile
   uint8_t* invs = l1s + kStages * p.l1_tile;
-  K1Shared* sh = reinterpret_cast<K1Shared*>(invs + kStages * kInvTile);
+  K1Shared* sh = reinterpret_cast<K1Shared*>(invs + kStages * kAux);
   float* red = reinterpret_cast<float*>(smem);  // reuses the stage buffers after the K loop
   const int red_stride = p.r_pad + 4;
 
@@ -122,6 +134,7 @@ __global__ void __launch_bounds__(kThreads, 2) act_quant_lowrank_kernel(
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sh->full[s], 1);
       mbar_init(&sh->empty[s], kQuantWarps + (lowrank ? 1 : 0));
+      mbar_init(&sh->normed[s], kQuantWarps);
     }
     mbar_init(&sh->tfull, 1);
     mbar_init(&sh->never, 1);
@@ -143,7 +156,7 @@ __global__ void __launch_bounds__(kThreads, 2) act_quant_lowrank_kernel(
     if (lane == 0) {
       tma_prefetch_desc(&map_x);
       if (lowrank) tma_prefetch_desc(&map_l1);
-      const uint32_t bytes = kXTile + (lowrank ? p.l1_tile : 0u) + kInvTile;
+      const uint32_t bytes = kXTile + (lowrank ? p.l1_tile : 0u) + kAux;
       int issued = 0;
       for (int i = 0; i < nt; ++i) {
         const int s = i % kStages;
@@ -153,7 +166,11 @@ __global__ void __launch_bounds__(kThreads, 2) act_quant_lowrank_kernel(
         const int k0 = (t0 + i) * 64;
         tma_load_2d(xs + s * kXTile, &map_x, &sh->full[s], k0, m0);
         if (lowrank) tma_load_2d(l1s + s * p.l1_tile, &map_l1, &sh->full[s], k0, 0);
-        bulk_load(invs + s * kInvTile, p.inv_lam + k0, kInvTile, &sh->full[s]);
+        bulk_load(invs + s * kAux, p.inv_lam + k0, kInvTile, &sh->full[s]);
+        if (kNorm) {
+          bulk_load(invs + s * kAux + kInvTile, p.norm_a + k0, kInvTile, &sh->full[s]);
+          bulk_load(invs + s * kAux + 2 * kInvTile, p.norm_c + k0, kInvTile, &sh->full[s]);
+        }
         issued = i + 1;
       }
       if (sh->abort) {  // let copies in flight land before the buffers are reused
@@ -167,7 +184,7 @@ __global__ void __launch_bounds__(kThreads, 2) act_quant_lowrank_kernel(
       for (int i = 0; i < nt; ++i) {
         const int s = i % kStages;
         const uint32_t ph = (i / kStages) & 1;
-        if (!wait_bounded(&sh->full[s], ph, wc)) break;
+        if (!wait_bounded(kNorm ? &sh->normed[s] : &sh->full[s], ph, wc)) break;  // X in the tile
         tc_fence_after();
         mma_bf16_x4(tmem, desc_kmajor_sw128(smem_u32(xs + s * kXTile)),
                     desc_kmajor_sw128(smem_u32(l1s + s * p.l1_tile)), idesc, i != 0);
@@ -181,13 +198,44 @@ __global__ void __launch_bounds__(kThreads, 2) act_quant_lowrank_kernel(
     const int row = 16 * wq + static_cast<int>(lane >> 1);
     const int h = lane & 1;                              // columns [32h, 32h + 32) of the tile
     const int m = m0 + row;
+    float mu = 0.0f, rstd = 0.0f;
+    if (kNorm && m < p.M) {
+      const float2 st = p.stats[m];
+      mu = st.x;
+      rstd = st.y;
+    }
     if (p.stall) wait_warp(&sh->never, 0, wc);
     for (int i = 0; i < nt; ++i) {
       const int s = i % kStages;
       const uint32_t ph = (i / kStages) & 1;
       if (!wait_warp(&sh->full[s], ph, wc)) break;
-      const uint8_t* xrow = xs + s * kXTile + row * 128;
-      const float4* inv4 = reinterpret_cast<const float4*>(invs + s * kInvTile) + 8 * h;
+      uint8_t* xrow = xs + s * kXTile + row * 128;
+      const float4* inv4 = reinterpret_cast<const float4*>(invs + s * kAux) + 8 * h;
+      if constexpr (kNorm) {
+        // z -> x = bf16(((z - mu) * rstd) * a + c) in place (zero on padding rows)
+        const float* na = reinterpret_cast<const float*>(invs + s * kAux + kInvTile) + 32 * h;
+        const float* nc = reinterpret_cast<const float*>(invs + s * kAux + 2 * kInvTile) + 32 * h;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint4* cp = reinterpret_cast<uint4*>(xrow + (((4 * h + c) ^ (row & 7)) << 4));
+          const uint4 z = *cp;
+          const uint32_t zw[4] = {z.x, z.y, z.z, z.w};
+          uint32_t xw[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j = 8 * c + 2 * e;
+            const float z0 = __uint_as_float(zw[e] << 16), z1 = __uint_as_float(zw[e] & 0xFFFF0000u);
+            const float x0 = __fadd_rn(__fmul_rn(__fmul_rn(__fsub_rn(z0, mu), rstd), na[j]), nc[j]);
+            const float x1 = __fadd_rn(__fmul_rn(__fmul_rn(__fsub_rn(z1, mu), rstd), na[j + 1]), nc[j + 1]);
+            const __nv_bfloat162 xb = __floats2bfloat162_rn(x0, x1);
+            xw[e] = m < p.M ? *reinterpret_cast<const uint32_t*>(&xb) : 0u;
+          }
+          *cp = make_uint4(xw[0], xw[1], xw[2], xw[3]);
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the MMA reads X through the async proxy
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh->normed[s]);
+      }
       const int kt = t0 + i;
       const int k0 = kt * 64;
       float v[32];
@@ -321,15 +369,22 @@ __global__ void __launch_bounds__(kThreads, 2) act_quant_lowrank_kernel(
   }
 }
 
+// The kernel instantiation for a format and front end.
+using K1Kernel = void (*)(const CUtensorMap, const CUtensorMap, const K1Params);
+K1Kernel k1_kernel(bool int4, bool norm) {
+  if (norm) return int4 ? act_quant_lowrank_kernel<true, true> : act_quant_lowrank_kernel<false, true>;
+  return int4 ? act_quant_lowrank_kernel<true, false> : act_quant_lowrank_kernel<false, false>;
+}
+
 // Clusters of this kernel that fit on the device at once for a K-split of S
 // (cluster = S CTAs); cached per (S, shared memory size).
-int max_active_clusters(int S, size_t smem, bool int4) {
+int max_active_clusters(int S, size_t smem, bool int4, bool norm) {
   static std::mutex mu;
   static std::map<std::pair<int, size_t>, int> cache;
   std::lock_guard<std::mutex> lk(mu);
   int dev = 0;
   cudaGetDevice(&dev);
-  const auto key = std::make_pair(S + 16 * dev + (int4 ? 4096 : 0), smem);
+  const auto key = std::make_pair(S + 64 * dev + (int4 ? 4096 : 0) + (norm ? 8192 : 0), smem);
   auto it = cache.find(key);
   if (it != cache.end()) return it->second;
   cudaLaunchConfig_t cfg = {};
@@ -344,8 +399,7 @@ int max_active_clusters(int S, size_t smem, bool int4) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  const cudaError_t qe = int4 ? cudaOccupancyMaxActiveClusters(&n, act_quant_lowrank_kernel<true>, &cfg)
-                              : cudaOccupancyMaxActiveClusters(&n, act_quant_lowrank_kernel<false>, &cfg);
+  const cudaError_t qe = cudaOccupancyMaxActiveClusters(&n, k1_kernel(int4, norm), &cfg);
   if (qe != cudaSuccess || n < 1) {
     cudaGetLastError();
     n = 1;
@@ -359,12 +413,12 @@ int max_active_clusters(int S, size_t smem, bool int4) {
 // placed one CTA per SM within a GPC, so splitting more only pays while the
 // clusters still fit: the cost is (waves of clusters) x (tiles per CTA), ties
 // going to the larger split (more CTAs in flight).  At least 4 tiles per CTA.
-int auto_splits(int mblocks, int kt_total, size_t smem, bool int4) {
+int auto_splits(int mblocks, int kt_total, size_t smem, bool int4, bool norm) {
   const int s_max = std::max(1, std::min(8, kt_total / 4));
   int best = 1;
   long best_cost = -1;
   for (int S = 1; S <= s_max; ++S) {
-    const int fit = max_active_clusters(S, smem, int4);
+    const int fit = max_active_clusters(S, smem, int4, norm);
     const long waves = (mblocks + fit - 1) / fit;
     const long cost = waves * ((kt_total + S - 1) / S);
     if (best_cost < 0 || cost <= best_cost) {
@@ -381,17 +435,19 @@ svdq_status launch_act_quant(const ActArgs& a, cudaStream_t stream) {
   const int mblocks = (a.M + 127) / 128;
   const int kt_total = a.K / 64;
   const uint32_t l1_tile = static_cast<uint32_t>(a.r_pad) * 128u;
-  const size_t smem = 1024 + kStages * (kXTile + l1_tile + kInvTile) + sizeof(K1Shared);
+  const bool norm = a.stats != nullptr;
+  const size_t smem = 1024 + kStages * (kXTile + l1_tile + kInvTile * (norm ? 3 : 1)) + sizeof(K1Shared);
   static bool attr_set[64] = {};  // per device: the attribute is set on the current one
   int cur_dev = 0;
   SVDQ_CUDA_TRY(cudaGetDevice(&cur_dev));
   if (cur_dev < 0 || cur_dev >= 64 || !attr_set[cur_dev]) {
-    SVDQ_CUDA_TRY(cudaFuncSetAttribute(act_quant_lowrank_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024));
-    SVDQ_CUDA_TRY(cudaFuncSetAttribute(act_quant_lowrank_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024));
+    for (int v = 0; v < 4; ++v)
+      SVDQ_CUDA_TRY(cudaFuncSetAttribute(k1_kernel(v & 1, v & 2), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         227 * 1024));
     if (cur_dev >= 0 && cur_dev < 64) attr_set[cur_dev] = true;
   }
   const int splits = a.splits > 0 ? std::min(std::min(a.splits, 8), kt_total)
-                                   : auto_splits(mblocks, kt_total, smem, a.int4 != 0);
+                                   : auto_splits(mblocks, kt_total, smem, a.int4 != 0, norm);
 
   CUtensorMap map_x;
   svdq_status st = make_tmap_2d(&map_x, a.X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.K, a.M,
@@ -413,6 +469,9 @@ svdq_status launch_act_quant(const ActArgs& a, cudaStream_t stream) {
   p.wait_ns = wait_limit_ns();
   p.stall = a.stall;
   p.m_pad = mblocks * 128;
+  p.stats = static_cast<const float2*>(a.stats);
+  p.norm_a = a.norm_a;
+  p.norm_c = a.norm_c;
   p.l1_tile = l1_tile;
   uint32_t cols = 32;
   while (cols < static_cast<uint32_t>(a.r_pad)) cols <<= 1;
@@ -431,10 +490,7 @@ svdq_status launch_act_quant(const ActArgs& a, cudaStream_t stream) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (a.int4)
-    SVDQ_CUDA_TRY(cudaLaunchKernelEx(&cfg, act_quant_lowrank_kernel<true>, map_x, map_l1, p));
-  else
-    SVDQ_CUDA_TRY(cudaLaunchKernelEx(&cfg, act_quant_lowrank_kernel<false>, map_x, map_l1, p));
+  SVDQ_CUDA_TRY(cudaLaunchKernelEx(&cfg, k1_kernel(a.int4 != 0, norm), map_x, map_l1, p));
   return SVDQ_OK;
 }
 

@@ -457,6 +457,36 @@ svdq_status svdq_quantize_act_lowrank_down(const svdq_weights* w, const void* X_
   return launch_act_quant(a, static_cast<cudaStream_t>(stream));
 }
 
+svdq_status svdq_act_row_stats(const void* Z_bf16, int M, int K, float eps, float* stats, void* stream) {
+  if (M < 1 || K < 64 || K % 64)
+    return fail(SVDQ_ERR_INVALID_ARG, "M=%d must be >= 1 and K=%d a positive multiple of 64", M, K);
+  if (!(eps >= 0.0f) || !std::isfinite(eps)) return fail(SVDQ_ERR_INVALID_ARG, "eps must be finite and >= 0");
+  SVDQ_TRY(check_dev_ptr(Z_bf16, "Z"));
+  SVDQ_TRY(check_dev_ptr(stats, "stats"));
+  SVDQ_TRY(check_device());
+  return launch_row_stats(Z_bf16, M, K, eps, stats, static_cast<cudaStream_t>(stream));
+}
+
+svdq_status svdq_norm_quantize_act_lowrank_down(const svdq_weights* w, const void* Z_bf16, int M, const float* stats,
+                                                const float* norm_a, const float* norm_c, void* xq, void* xsf,
+                                                void* T, void* stream) {
+  SVDQ_TRY(check_runtime(w, M));
+  SVDQ_TRY(check_dev_ptr(Z_bf16, "Z"));
+  SVDQ_TRY(check_dev_ptr(stats, "stats"));
+  SVDQ_TRY(check_dev_ptr(norm_a, "norm_a"));
+  SVDQ_TRY(check_dev_ptr(norm_c, "norm_c"));
+  SVDQ_TRY(check_dev_ptr(xq, "xq"));
+  SVDQ_TRY(check_dev_ptr(xsf, "xsf"));
+  if (w->r_pad > 0) SVDQ_TRY(check_dev_ptr(T, "T"));
+  ActArgs a{M, w->K, w->r_pad, Z_bf16, &w->map_l1, w->d_inv_lam, static_cast<uint8_t*>(xq),
+            static_cast<uint8_t*>(xsf), static_cast<uint16_t*>(T), 0, 0};
+  a.int4 = w->format == SVDQ_FORMAT_INT4;
+  a.stats = stats;
+  a.norm_a = norm_a;
+  a.norm_c = norm_c;
+  return launch_act_quant(a, static_cast<cudaStream_t>(stream));
+}
+
 svdq_status svdq_debug_launch_stalled_act(const svdq_weights* w, const void* X_bf16, int M, void* xq, void* xsf,
                                           void* T, void* stream) {
   SVDQ_TRY(check_runtime(w, M));
@@ -526,6 +556,10 @@ size_t svdq_forward_workspace_bytes(const svdq_weights* w, int M) {
   return up256(svdq_act_codes_bytes(M, w->K)) + up256(svdq_act_sf_bytes(M, w->K)) +
          up256(svdq_lowrank_bytes(w, M));
 }
+size_t svdq_forward_norm_workspace_bytes(const svdq_weights* w, int M) {
+  if (!w || M < 1) return 0;
+  return svdq_forward_workspace_bytes(w, M) + up256(static_cast<size_t>(M) * 8);
+}
 size_t svdq_forward_host_workspace_bytes(const svdq_weights* w, int M) {
   if (!w || M < 1) return 0;
   return svdq_forward_workspace_bytes(w, M) + up256(static_cast<size_t>(M) * w->K * 2) +
@@ -544,6 +578,25 @@ svdq_status svdq_forward(const svdq_weights* w, const void* X_bf16, int M, void*
   uint8_t* xsf = xq + up256(svdq_act_codes_bytes(M, w->K));
   uint8_t* T = xsf + up256(svdq_act_sf_bytes(M, w->K));
   SVDQ_TRY(svdq_quantize_act_lowrank_down(w, X_bf16, M, xq, xsf, w->r_pad ? T : nullptr, stream));
+  return svdq_linear_w4a4(w, xq, xsf, w->r_pad ? T : nullptr, M, Y_bf16, stream);
+}
+
+svdq_status svdq_forward_norm(const svdq_weights* w, const void* Z_bf16, int M, const float* norm_a,
+                              const float* norm_c, float eps, void* Y_bf16, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+  SVDQ_TRY(check_runtime(w, M));
+  SVDQ_TRY(check_dev_ptr(workspace, "workspace"));
+  if (workspace_bytes < svdq_forward_norm_workspace_bytes(w, M))
+    return fail(SVDQ_ERR_INVALID_ARG, "workspace has %zu bytes, needs %zu", workspace_bytes,
+                svdq_forward_norm_workspace_bytes(w, M));
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint8_t* xq = ws;
+  uint8_t* xsf = xq + up256(svdq_act_codes_bytes(M, w->K));
+  uint8_t* T = xsf + up256(svdq_act_sf_bytes(M, w->K));
+  float* stats = reinterpret_cast<float*>(ws + svdq_forward_workspace_bytes(w, M));
+  SVDQ_TRY(svdq_act_row_stats(Z_bf16, M, w->K, eps, stats, stream));
+  SVDQ_TRY(svdq_norm_quantize_act_lowrank_down(w, Z_bf16, M, stats, norm_a, norm_c, xq, xsf, w->r_pad ? T : nullptr,
+                                               stream));
   return svdq_linear_w4a4(w, xq, xsf, w->r_pad ? T : nullptr, M, Y_bf16, stream);
 }
 

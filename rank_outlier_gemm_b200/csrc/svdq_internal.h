@@ -57,8 +57,13 @@ struct ActArgs {
   int splits;               // K-splits per 128-row block (0 = automatic)
   int* err = nullptr;       // device error word (nullptr = the device's default word)
   int int4 = 0;             // INT4 variant: group-64 codes, bf16 scales [K/64][rows padded to 128]
+  const void* stats = nullptr;   // norm front end: device (mu, rstd) per row; X is then the pre-norm Z
+  const float* norm_a = nullptr;  // norm front end: device per-channel multiplier [K]
+  const float* norm_c = nullptr;  // norm front end: device per-channel offset [K]
 };
 svdq_status launch_act_quant(const ActArgs& a, cudaStream_t stream);
+// Per-row LayerNorm statistics (mu, rstd) of a device bf16 [M, K] array into device float [M][2].
+svdq_status launch_row_stats(const void* Z, int M, int K, float eps, float* stats, cudaStream_t stream);
 
 struct GemmArgs {
   int M, N, K, r_pad;
