@@ -329,6 +329,38 @@ def int4_layers(L, torch, layers, dev, stream, reps=30):
     return out
 
 
+def norm_fusion(L, torch, layers, dev, stream, reps=30, eps=1e-6):
+    """NEXT-3, the activation kernel fused with the adaLN front end (LayerNorm
+    over K, then a = 1 + scale, c = shift per channel): per step layer, the
+    fused path (row statistics + fused activation kernel + GEMM) against the
+    unfused one (a PyTorch LayerNorm and modulation writing bf16 X, then the
+    layer), and the layer alone on a ready X for reference."""
+    out = {}
+    g = torch.Generator(device="cpu").manual_seed(5)
+    for l in layers:
+        c, w = l["case"], l["w"]
+        Z = (torch.randn(c.M, c.K, generator=g) * 2 + 1).to(torch.bfloat16).to(dev)
+        a = (1 + 0.1 * torch.randn(c.K, generator=g)).to(dev)
+        sh = (0.1 * torch.randn(c.K, generator=g)).to(dev)
+        ws = torch.empty(L.svdq_forward_norm_workspace_bytes(w, c.M), dtype=torch.uint8, device=dev)
+        Y = l["Y"]
+
+        def fused():
+            L.svdq_forward_norm(w, Z, a, sh, eps, Y, ws)
+
+        def unfused():
+            X = (torch.nn.functional.layer_norm(Z.float(), (c.K,), eps=eps) * a + sh).to(torch.bfloat16)
+            L.svdq_forward(w, X, Y, ws)
+
+        def layer_only():
+            L.svdq_forward(w, l["X"], Y, ws)
+
+        out[c.name] = {"fused_us": 1e3 * _time_ms(torch, stream, fused, reps),
+                       "unfused_us": 1e3 * _time_ms(torch, stream, unfused, reps),
+                       "layer_only_us": 1e3 * _time_ms(torch, stream, layer_only, reps)}
+    return out
+
+
 def alpha_search(L, rows=256):
     """NEXT-3 (App. D migration strength): relative output error per candidate
     alpha on a calibration batch of one FLUX layer, through the library's own
@@ -441,7 +473,7 @@ def run_ours(args):
 
     # low-rank overhead: the same kernels at rank 0 (extras)
     overhead = None
-    unfused = sweep = small = refine = asearch = int4 = None
+    unfused = sweep = small = refine = asearch = int4 = normf = None
     if args.extras:
         def step0():
             for l in layers:
@@ -467,6 +499,7 @@ def run_ours(args):
             refine = refinement(L)
             asearch = alpha_search(L)
             int4 = int4_layers(L, torch, layers, dev, stream) if args.format == "nvfp4" else None
+            normf = norm_fusion(L, torch, layers, dev, stream)
 
     # end to end through the public host-buffer call: H2D of X, both kernels, D2H of Y
     e2e = None
@@ -526,6 +559,7 @@ def run_ours(args):
             "refinement": refine,
             "alpha_search": asearch,
             "int4": int4,
+            "norm_fusion": normf,
             "gpu_launches": 2 * nl * args.steps,
             "e2e": e2e,
         }

@@ -252,8 +252,10 @@ svdq_status svdq_norm_quantize_act_lowrank_down(const svdq_weights* w, const voi
 
 /*
  * LayerNorm statistics per token: mu = mean_j z_j and
- * rstd = 1 / sqrt(mean_j (z_j - mu)^2 + eps), accumulated in fp32 (two passes
- * over the row), IEEE square root and reciprocal.
+ * rstd = 1 / sqrt(mean_j (z_j - mu)^2 + eps), in one read of the row: fp32 sums
+ * of d = z - z0 and d^2 (z0 = the row's first value, so the one-pass variance
+ * E[d^2] - E[d]^2 does not cancel for a mean far from zero), IEEE square root
+ * and reciprocal.
  *   Z_bf16  device, M x K bf16;  stats  device, M x 2 floats (out)
  * SVDQ_ERR_INVALID_ARG for bad sizes, eps < 0 or misaligned pointers.
  */

@@ -3,10 +3,11 @@
 // The configured DiT blocks feed their linear layers adaLN(z) = (1 + scale) *
 // LayerNorm(z) + shift; the activation kernel applies that per element and
 // needs mu and rstd of each token over its K channels first.  One warp per
-// row: a pass for the mean and a second pass (mostly from L2) for the centred
-// sum of squares, both accumulated in fp32 per lane and combined by a fixed
-// shuffle tree; rstd = 1 / sqrt(var + eps) with IEEE square root and
-// reciprocal.
+// row and one read of it: each lane accumulates, in fp32, the sum and the sum
+// of squares of d = z - z0, with z0 the row's first value (a shift that keeps
+// the one-pass variance E[d^2] - E[d]^2 from cancelling when the mean is far
+// from zero); a fixed shuffle tree combines the lanes; mu = z0 + E[d] and
+// rstd = 1 / sqrt(var + eps) with IEEE square root and reciprocal.
 #include "ptx.cuh"
 #include "svdq_internal.h"
 
@@ -31,22 +32,23 @@ __global__ void __launch_bounds__(32 * kRowsPerBlock) row_stats_kernel(const uin
   if (m >= M) return;
   const uint4* row = reinterpret_cast<const uint4*>(Z + static_cast<size_t>(m) * K);
   const int n8 = K / 8;  // 16-byte chunks of 8 values
-  float s = 0.0f;
+  const float z0 = __uint_as_float(static_cast<uint32_t>(__ldg(Z + static_cast<size_t>(m) * K)) << 16);
+  float s1 = 0.0f, s2 = 0.0f;
+#pragma unroll 4
   for (int i = lane; i < n8; i += 32) {
     const uint4 w = __ldg(row + i);
-    s += bf16_lo(w.x) + bf16_hi(w.x) + bf16_lo(w.y) + bf16_hi(w.y) + bf16_lo(w.z) + bf16_hi(w.z) +
-         bf16_lo(w.w) + bf16_hi(w.w);
-  }
-  const float mu = __fdiv_rn(warp_sum(s), static_cast<float>(K));
-  float q = 0.0f;
-  for (int i = lane; i < n8; i += 32) {
-    const uint4 w = __ldg(row + i);
-    const float d[8] = {bf16_lo(w.x) - mu, bf16_hi(w.x) - mu, bf16_lo(w.y) - mu, bf16_hi(w.y) - mu,
-                        bf16_lo(w.z) - mu, bf16_hi(w.z) - mu, bf16_lo(w.w) - mu, bf16_hi(w.w) - mu};
+    const float d[8] = {bf16_lo(w.x) - z0, bf16_hi(w.x) - z0, bf16_lo(w.y) - z0, bf16_hi(w.y) - z0,
+                        bf16_lo(w.z) - z0, bf16_hi(w.z) - z0, bf16_lo(w.w) - z0, bf16_hi(w.w) - z0};
+    s1 += ((d[0] + d[1]) + (d[2] + d[3])) + ((d[4] + d[5]) + (d[6] + d[7]));
+    float q = 0.0f;
 #pragma unroll
     for (int j = 0; j < 8; ++j) q = __fmaf_rn(d[j], d[j], q);
+    s2 += q;
   }
-  const float var = __fdiv_rn(warp_sum(q), static_cast<float>(K));
+  const float inv_k = 1.0f / static_cast<float>(K);
+  const float m1 = warp_sum(s1) * inv_k;
+  const float var = fmaxf(warp_sum(s2) * inv_k - m1 * m1, 0.0f);
+  const float mu = z0 + m1;
   if (lane == 0) stats[m] = make_float2(mu, __frcp_rn(__fsqrt_rn(__fadd_rn(var, eps))));
 }
 
