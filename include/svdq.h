@@ -377,7 +377,8 @@ svdq_status svdq_debug_launch_stalled_act(const svdq_weights* w, const void* X_b
  * Test hook: svdq_linear_w4a4 with the split-K factor fixed to `ksplit` CTAs
  * per output tile (1 = no split) instead of the automatic choice.  The split
  * is clamped to the number of 256-wide K tiles; a split whose clusters would
- * not all be resident at once falls back to 1.  SVDQ_ERR_INVALID_ARG unless
+ * not all be resident at once falls back to 1.  INT4 handles have no split-K:
+ * for them the call is svdq_linear_w4a4.  SVDQ_ERR_INVALID_ARG unless
  * 1 <= ksplit <= 8; otherwise as svdq_linear_w4a4.
  */
 svdq_status svdq_debug_linear_w4a4_ksplit(const svdq_weights* w, const void* xq, const void* xsf,

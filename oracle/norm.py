@@ -3,8 +3,8 @@
 TEST INFRASTRUCTURE ONLY: part of the CPU oracle (see ``oracle/__init__.py``).
 
 SVDQuant (paperlayer.ai summary of arXiv 2411.05007v4), §4.3: the down-projection
-shares the activation read with the quantization kernel; the survey's NEXT-3
-also fuses that kernel into the norm ahead of the layer.  In the DiT blocks of
+shares the activation read with the quantization kernel; the fused path here
+carries that one step further, into the norm ahead of the layer.  In the DiT blocks of
 the configured models the linear layers read LayerNorm(z) modulated per channel
 (adaLN: (1 + scale) * LN(z) + shift), so the fused input is
 

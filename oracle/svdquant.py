@@ -167,7 +167,7 @@ def prepare(W, act_absmax, bias, rank: int, alpha: float = 0.5, iters: int = 1) 
 
 def search_alpha(W, X, bias, rank: int, alphas, iters: int = 1):
     """Per-layer smoothing strength (App. D: alpha is the migration strength of
-    the smoothing; the survey's NEXT-3 reading): for each candidate, prepare
+    the smoothing; choosing it per layer this way is a reading): for each candidate, prepare
     with the calibration batch's per-channel maxima and score the layer output
     by ||Y - (X W^T + b)||_F / ||X W^T + b||_F in float64.  Returns (errors,
     index of the smallest)."""

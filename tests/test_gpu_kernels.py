@@ -327,7 +327,7 @@ def test_library_prepare_invariants():
 
 
 def test_library_refinement_matches_oracle():
-    """Refined split (SVDQuant §4.2, the survey's reading of its iterations):
+    """Refined split (SVDQuant §4.2; the update rule is a reading of its iterations):
     the library's residual quantization errors follow the oracle's (exact SVD)
     closely, the kept split is the one with the smallest error (recomputed by
     the oracle from the exported residual), refinement lowers the error on the
