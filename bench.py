@@ -61,10 +61,10 @@ def peaks():
 # kernel source the counters were taken on; counters of another source are stale
 # and not reported.
 K2_TRAFFIC = {
-    "source_sha256": "11554d84cb53683ba96d19403a047117614bfa2844fec6ffc17f189da222e94f",
+    "source_sha256": "4aaa299b83115cf162973296dfe5b0fff5da7d2f120f9935a301ac7e05427a3e",
     # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum: read + write per launch
-    "bytes_per_launch": {"attn_out": 14110464 + 1792, "qkv": 25147648 + 32385280,
-                         "mlp_up": 30663680 + 59214336, "mlp_down": 56352512 + 6549248},
+    "bytes_per_launch": {"attn_out": 14127104 + 16384, "qkv": 25167104 + 32058880,
+                         "mlp_up": 30682112 + 59258624, "mlp_down": 55453440 + 5070592},
 }
 
 
@@ -361,6 +361,56 @@ def norm_fusion(L, torch, layers, dev, stream, reps=30, eps=1e-6):
     return out
 
 
+def _cublaslt_fp4_us(torch, M, K, N, dev, stream, reps):
+    """cuBLASLt's NVFP4 GEMM (torch._scaled_mm on float4_e2m1fn_x2 with E4M3 block
+    scales in the 128 x 4 atom layout, bf16 out, no low-rank branch): a plain
+    library GEMM timed only as a measured FP4 reference; None when this torch
+    build has no such path."""
+    if not hasattr(torch, "float4_e2m1fn_x2"):
+        return None
+    g = torch.Generator(device=dev).manual_seed(0)
+
+    def atoms(rows):
+        kb = K // 16
+        return torch.full((((rows + 127) // 128 * 128) * kb,), 0x30, dtype=torch.uint8,
+                          device=dev).view(torch.float8_e4m3fn)  # 0x30 = 0.5, every block
+
+    a = torch.randint(0, 256, (M, K // 2), dtype=torch.uint8, device=dev, generator=g).view(torch.float4_e2m1fn_x2)
+    b = torch.randint(0, 256, (N, K // 2), dtype=torch.uint8, device=dev, generator=g).view(torch.float4_e2m1fn_x2)
+    sa, sb = atoms(M), atoms(N)
+    try:
+        return 1e3 * _time_ms(torch, stream, lambda: torch._scaled_mm(a, b.t(), sa, sb, out_dtype=torch.bfloat16),
+                              reps)
+    except (RuntimeError, TypeError) as ex:  # no NVFP4 kernel in this build
+        print(f"cuBLASLt NVFP4 GEMM unavailable: {str(ex)[:200]}", file=sys.stderr)
+        return None
+
+
+def fp4_reference(L, torch, dev, stream, reps=20):
+    """A measured FP4 rate beside the nominal one: this library's GEMM (rank 0,
+    unit smoothing, random weights and activations) and cuBLASLt's NVFP4 GEMM on
+    a large square problem and on the step's largest layer shape, as TFLOP/s."""
+    out = {}
+    for name, (M, K, N) in {"square_8192": (8192, 8192, 8192), "flux_mlp_up": (4608, 3072, 12288)}.items():
+        rng = np.random.default_rng(M + K + N)
+        R = rng.standard_normal((N, K), dtype=np.float32) * np.float32(0.02)
+        w = L.svdq_weights_from_factors(N, K, 0, np.ones(K, np.float32), None, None, R)
+        del R
+        X = torch.randn((M, K), generator=torch.Generator(device=dev).manual_seed(1), device=dev).to(torch.bfloat16)
+        xq, xsf, _ = L.act_buffers(w, M, dev)
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        L.svdq_quantize_act_lowrank_down(w, X, xq, xsf, None)
+        us = 1e3 * _time_ms(torch, stream, lambda: L.svdq_linear_w4a4(w, xq, xsf, None, M, Y), reps)
+        del X
+        cub = _cublaslt_fp4_us(torch, M, K, N, dev, stream, reps)
+        fl = 2.0 * M * N * K
+        out[name] = {"M": M, "K": K, "N": N, "ours_us": us, "ours_tflops": fl / (us * 1e-6) / 1e12,
+                     "cublaslt_us": cub, "cublaslt_tflops": fl / (cub * 1e-6) / 1e12 if cub else None}
+        del w, xq, xsf, Y
+        torch.cuda.empty_cache()
+    return out
+
+
 def alpha_search(L, rows=256):
     """NEXT-3 (App. D migration strength): relative output error per candidate
     alpha on a calibration batch of one FLUX layer, through the library's own
@@ -473,7 +523,7 @@ def run_ours(args):
 
     # low-rank overhead: the same kernels at rank 0 (extras)
     overhead = None
-    unfused = sweep = small = refine = asearch = int4 = normf = None
+    unfused = sweep = small = refine = asearch = int4 = normf = fp4ref = None
     if args.extras:
         def step0():
             for l in layers:
@@ -500,6 +550,7 @@ def run_ours(args):
             asearch = alpha_search(L)
             int4 = int4_layers(L, torch, layers, dev, stream) if args.format == "nvfp4" else None
             normf = norm_fusion(L, torch, layers, dev, stream)
+            fp4ref = fp4_reference(L, torch, dev, stream) if args.format == "nvfp4" else None
 
     # end to end through the public host-buffer call: H2D of X, both kernels, D2H of Y
     e2e = None
@@ -560,6 +611,7 @@ def run_ours(args):
             "alpha_search": asearch,
             "int4": int4,
             "norm_fusion": normf,
+            "fp4_reference": fp4ref,
             "gpu_launches": 2 * nl * args.steps,
             "e2e": e2e,
         }

@@ -17,7 +17,9 @@
 //   warps 2-5  scale writers: read the scale atoms of a K tile from shared
 //              memory and write them into TMEM with tcgen05.st, replicated into
 //              each 32-lane quarter (the layout the block-scaled MMA reads)
-//   warps 6-9  epilogue: tcgen05.ld, y = alpha_w*acc + b, bf16 RNE, 16-byte stores
+//   warps 6-9  epilogue: tcgen05.ld, y = alpha_w*acc + b, bf16 RNE; 32 x 32
+//              chunks staged in shared memory and written by TMA stores while
+//              a long main loop follows, stored from registers otherwise
 // TMEM (512 columns) holds two 256-column accumulators.  Tile j accumulates in
 // acc[j%2] and keeps its scale slots (2 x 48 columns, one K tile each) in the first 96 columns
 // of acc[(j+1)%2], which the epilogue of tile j-1 releases first; so the
@@ -73,13 +75,16 @@ struct K2Params {
   const float* bias;
   float alpha_w;
   uint16_t* Y;
-  int y32;         // Y is 32-byte aligned: one 32-byte store per 16 columns
+  int y32;         // Y is 32-byte aligned: one 32-byte store per 16 columns (direct stores)
+  int tma_y;       // tiles long enough to hide a staged epilogue use TMA stores of Y
   int* err;
   uint64_t wait_ns;
 };
 
 struct K2Shared {
-  alignas(16) float bias[4][kBN];  // one slice per epilogue warp (read as float4)
+  // one 32 x 32 bf16 chunk of Y per epilogue warp, in the 64-byte-swizzled
+  // layout of the Y tensor map
+  alignas(1024) uint8_t ystage[4][2048];
   uint64_t full[kStages];
   uint64_t empty[kStages];
   uint64_t sf_full[kSfSlots];
@@ -106,18 +111,15 @@ __device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// y = alpha_w * acc + b for 32 consecutive columns of one row, bf16 RNE.  alpha_w
-// is a power of two, so alpha_w * acc is exact (outside the subnormal range) and
-// one fused multiply-add rounds exactly like the product followed by the sum.
-// Each lane writes whole 32-byte sectors when Y allows it (else 16-byte halves).
-__device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], const float* bias_s, const K2Params& p,
-                                            int m, int n) {
-  if (m >= p.M || n >= p.N) return;
-  uint32_t packed[16];
-  const float4* b4 = reinterpret_cast<const float4*>(bias_s);
+// y = alpha_w * acc + b for 32 consecutive columns of one row, bf16 RNE, packed
+// in pairs.  alpha_w is a power of two, so alpha_w * acc is exact (outside the
+// subnormal range) and one fused multiply-add rounds exactly like the product
+// followed by the sum.
+__device__ __forceinline__ void epi_pack(const uint32_t (&r)[32], const K2Params& p, int n, uint32_t (&packed)[16]) {
+  const float4* b4 = reinterpret_cast<const float4*>(p.bias + n);  // padded to a multiple of 256
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const float4 bv = b4[i];
+    const float4 bv = __ldg(b4 + i);
     const float y0 = __fmaf_rn(__uint_as_float(r[4 * i + 0]), p.alpha_w, bv.x);
     const float y1 = __fmaf_rn(__uint_as_float(r[4 * i + 1]), p.alpha_w, bv.y);
     const float y2 = __fmaf_rn(__uint_as_float(r[4 * i + 2]), p.alpha_w, bv.z);
@@ -125,6 +127,43 @@ __device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], const float
     packed[2 * i] = bf16x2_rn(y0, y1);
     packed[2 * i + 1] = bf16x2_rn(y2, y3);
   }
+}
+
+// One 32 x 32 chunk of the warp's rows (row `lane`, 32 columns per lane) to Y
+// through the warp's staging buffer and one TMA store: four conflict-free
+// 16-byte shared stores per lane instead of 32 scattered row segments per
+// global store instruction, which keeps the epilogue's traffic off the load /
+// store pipe the main loop's shared-memory accesses share.  The store clips rows
+// >= M; its issue waits for the previous chunk's store to read the buffer, so a
+// chunk takes longer than a direct store: used while the next tile's main loop
+// is long enough to hide it.
+__device__ __forceinline__ void store_chunk_tma(const uint32_t (&r)[32], const K2Params& p, const CUtensorMap* map_y,
+                                                uint8_t* stage, uint32_t lane, int m_warp, int n) {
+  if (m_warp >= p.M || n >= p.N) return;
+  uint32_t packed[16];
+  epi_pack(r, p, n, packed);
+  if (lane == 0) bulk_wait_read<0>();  // the previous chunk's store has read the buffer
+  __syncwarp();
+  // 64-byte rows, 64-byte swizzle: row r's 16-byte piece i sits at piece i ^ ((r >> 1) & 3)
+  uint4* row = reinterpret_cast<uint4*>(stage + lane * 64);
+  const uint32_t sw = (lane >> 1) & 3u;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    row[i ^ sw] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(map_y, stage, n, m_warp);
+    bulk_commit_group();
+  }
+}
+
+// The same chunk stored straight from registers: each lane writes its row's 64
+// bytes as whole 32-byte sectors when Y allows it (else 16-byte halves).
+__device__ __forceinline__ void store_chunk_direct(const uint32_t (&r)[32], const K2Params& p, int m, int n) {
+  if (m >= p.M || n >= p.N) return;
+  uint32_t packed[16];
+  epi_pack(r, p, n, packed);
   uint16_t* dst = p.Y + static_cast<size_t>(m) * p.N + n;
   if (p.y32) {
 #pragma unroll
@@ -136,6 +175,41 @@ __device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], const float
       if (n + 8 * i < p.N)
         *reinterpret_cast<uint4*>(dst + 8 * i) =
             make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+  }
+}
+
+// One warp's share of a tile's epilogue (its 32 rows, 256 columns): chunks 0-2
+// first, whose accumulator columns then take the next tile's scale slots, then
+// chunks 3-7, each chunk's TMEM load in flight while the one before is stored.
+template <bool kTma>
+__device__ __forceinline__ void epilogue_tile(const K2Params& p, const CUtensorMap* map_y, uint32_t acc,
+                                              uint64_t* sfreg_free, uint8_t* ys, uint32_t lane, int m_warp, int n0) {
+  auto put = [&](const uint32_t(&rr)[32], int c) {
+    if constexpr (kTma)
+      store_chunk_tma(rr, p, map_y, ys, lane, m_warp, n0 + 32 * c);
+    else
+      store_chunk_direct(rr, p, m_warp + static_cast<int>(lane), n0 + 32 * c);
+  };
+  uint32_t r[3][32];
+#pragma unroll
+  for (int c = 0; c < 3; ++c) tmem_ld_x32(acc + 32 * c, r[c]);
+  tmem_ld_wait();
+  // columns 0..95 read: the next tile's scale slots may go there
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(sfreg_free);
+  uint32_t nx[32];
+  tmem_ld_x32(acc + 96, nx);
+#pragma unroll
+  for (int c = 0; c < 3; ++c) put(r[c], c);
+#pragma unroll
+  for (int c = 3; c < kBN / 32; ++c) {
+    tmem_ld_wait_regs(nx);
+    uint32_t cur[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) cur[i] = nx[i];
+    if (c + 1 < kBN / 32) tmem_ld_x32(acc + 32 * (c + 1), nx);
+    put(cur, c);
   }
 }
 
@@ -175,11 +249,12 @@ __device__ __forceinline__ void split_reduce(const K2Params& p, const float* par
 __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
     const __grid_constant__ CUtensorMap map_xq, const __grid_constant__ CUtensorMap map_wq,
     const __grid_constant__ CUtensorMap map_t, const __grid_constant__ CUtensorMap map_l2,
+    const __grid_constant__ CUtensorMap map_y,
     const K2Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   K2Shared* sh = reinterpret_cast<K2Shared*>(smem + kStages * kStage);
-  static_assert(offsetof(K2Shared, bias) % 16 == 0, "bias slices are read as float4");
+  static_assert(offsetof(K2Shared, ystage) == 0, "Y staging buffers keep the 1024-byte alignment the swizzle needs");
   static_assert((kStages * kStage) % 1024 == 0, "stage buffers keep 1024-byte alignment");
 
   const uint32_t warp = warp_id(), lane = lane_id();
@@ -441,20 +516,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
     const int q = warp & 3;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     const int row = q * 32 + lane;
+    uint8_t* ys = sh->ystage[warp - 6];
     int j = 0;
     for (int t = tile0; t < ntiles_total; t += tile_step, ++j) {
       const int a = j & 1;
-      const int m = (t % p.mtiles) * 128 + row;
+      const int m_warp = (t % p.mtiles) * 128 + q * 32;
+      const int m = m_warp + static_cast<int>(lane);
       const int n0 = (t / p.mtiles) * kBN;
-      // stage this tile's bias slice (per warp) while the main loop still runs
-      float* bias_s = sh->bias[warp - 6];
-      {
-        const float4* src = reinterpret_cast<const float4*>(p.bias + n0) + 2 * lane;
-        float4* dstb = reinterpret_cast<float4*>(bias_s) + 2 * lane;
-        dstb[0] = __ldg(src);
-        dstb[1] = __ldg(src + 1);
-      }
-      __syncwarp();
+      // staged TMA stores while another tile's main loop follows; the CTA's last
+      // tile (nothing left to overlap) and short tiles store directly
+      const bool tma = p.tma_y && t + tile_step < ntiles_total;
       if (!wait_warp(&sh->acc_full[a], (j >> 1) & 1, wc)) break;
       tc_fence_after();
       if (S > 1) {
@@ -481,26 +552,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
         }
         continue;
       }
-      uint32_t r[3][32];
-#pragma unroll
-      for (int c = 0; c < 3; ++c) tmem_ld_x32(tmem + a * 256 + lane_off + 32 * c, r[c]);
-      tmem_ld_wait();
-      // columns 0..95 read: the next tile's scale slots may go there
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sh->sfreg_free[a]);
-#pragma unroll
-      for (int c = 0; c < 3; ++c) store_chunk(r[c], bias_s + 32 * c, p, m, n0 + 32 * c);
-      for (int c = 3; c < kBN / 32; ++c) {
-        uint32_t rr[32];
-        tmem_ld_x32(tmem + a * 256 + lane_off + 32 * c, rr);
-        tmem_ld_wait();
-        store_chunk(rr, bias_s + 32 * c, p, m, n0 + 32 * c);
-      }
+      if (tma)
+        epilogue_tile<true>(p, &map_y, tmem + a * 256 + lane_off, &sh->sfreg_free[a], ys, lane, m_warp, n0);
+      else
+        epilogue_tile<false>(p, &map_y, tmem + a * 256 + lane_off, &sh->sfreg_free[a], ys, lane, m_warp, n0);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh->acc_empty[a]);
     }
+    if (lane == 0) bulk_wait_all();  // Y written, the staging buffer no longer read
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -599,6 +660,8 @@ svdq_status launch_gemm_w4a4(const GemmArgs& a, cudaStream_t stream) {
   p.Y = static_cast<uint16_t*>(a.Y);
   // N % 16 == 0, so every 16-column piece starts 32 bytes after the last
   p.y32 = (reinterpret_cast<uintptr_t>(a.Y) & 31u) == 0;
+  // a tile of at least 8 K steps (K >= 1792) hides the staged epilogue of the one before
+  p.tma_y = p.kt + p.slab >= 8 ? 1 : 0;
   p.err = a.err ? a.err : device_error_word();
   p.wait_ns = wait_limit_ns();
   if (!p.err) return fail(SVDQ_ERR_CUDA, "device error word unavailable");
@@ -614,6 +677,11 @@ svdq_status launch_gemm_w4a4(const GemmArgs& a, cudaStream_t stream) {
     if (st != SVDQ_OK) return st;
   }
   const CUtensorMap& map_l2 = a.r_pad > 0 ? *a.map_l2_256 : map_xq;
+  // Y in 32 x 32 boxes (64-byte rows, 64-byte swizzle) for the epilogue's stores
+  CUtensorMap map_y;
+  st = make_tmap_2d(&map_y, a.Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.N, a.M, static_cast<uint64_t>(a.N) * 2, 32, 32,
+                    CU_TENSOR_MAP_SWIZZLE_64B);
+  if (st != SVDQ_OK) return st;
 
   const size_t smem = 1024 + static_cast<size_t>(kStages) * kStage + sizeof(K2Shared);
   static bool attr_set[64] = {};  // per device: the attribute is set on the current one
@@ -645,7 +713,7 @@ svdq_status launch_gemm_w4a4(const GemmArgs& a, cudaStream_t stream) {
   attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = p.ksplit > 1 ? 2 : 1;
-  SVDQ_CUDA_TRY(cudaLaunchKernelEx(&cfg, gemm_w4a4_kernel, map_xq, *a.map_wq_256, map_t, map_l2, p));
+  SVDQ_CUDA_TRY(cudaLaunchKernelEx(&cfg, gemm_w4a4_kernel, map_xq, *a.map_wq_256, map_t, map_l2, map_y, p));
   return SVDQ_OK;
 }
 
