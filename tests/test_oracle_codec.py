@@ -76,6 +76,42 @@ def test_scale_is_rne_of_amax_over_qmax():
     np.testing.assert_array_equal(F.e4m3_decode(scales.reshape(-1)), ref)
 
 
+def test_scale_on_e4m3_midpoints():
+    """The scale is E4M3_RNE of the correctly rounded quotient amax / 6, worked
+    at the places where a slip shows.  amax = 6.375: the quotient 1.0625 is
+    exact and halfway between the E4M3 values 1.0 and 1.125; the tie goes to the
+    even mantissa, 1.0 (byte 0x38), so a scale nudged upward first would give
+    1.125.  amax = 7.1249995 (0x40E3FFFF, one ulp below 7.125): the exact
+    quotient is 1.1875 - 7.9e-8, which rounds to the fp32 value one ulp (1.2e-7)
+    below the 1.125 / 1.25 midpoint 1.1875, so the scale is 1.125 (0x39);
+    multiplying by fp32(1/6) = 1/6 + 5.0e-9 instead lands on 1.1875 itself and
+    the tie would give 1.25."""
+    g = np.zeros((2, 16), np.float32)
+    g[0, 3] = 6.375
+    g[1, 0] = np.array([0x40E3FFFF], np.uint32).view(np.float32)[0]
+    _, scales = C.quantize_groups(g)
+    np.testing.assert_array_equal(scales[:, 0], [0x38, 0x39])
+
+
+def test_codes_multiply_by_the_reciprocal_of_the_scale():
+    """Reading of the codec step: v' = fp32(v * fp32(1/s)).  A worked group where
+    it differs from dividing by s: amax = 10.5 gives s = 10.5 / 6 = 1.75 (exact,
+    E4M3 byte 0x3E) and fp32(1/1.75) = 4/7 + 2.6e-8.  For v = 3.0624998
+    (0x4043FFFF, one ulp below 3.0625 = 1.75 * 1.75) the product is
+    1.75 - 5.8e-8, within half an ulp (6.0e-8) of 1.75, so v' = 1.75 exactly,
+    the E2M1 midpoint of 1.5 and 2.0, and the tie gives 2.0 (code 4); v / s
+    would be 1.75 - 1.4e-7, which rounds below the midpoint to 1.5 (code 3).
+    10.5 itself becomes 10.5 * fp32(1/1.75) = 6.0000005, saturated to 6 (code 7)."""
+    g = np.zeros((1, 16), np.float32)
+    g[0, 0] = 10.5
+    g[0, 1] = np.array([0x4043FFFF], np.uint32).view(np.float32)[0]
+    g[0, 2] = -g[0, 1]
+    codes, scales = C.quantize_groups(g)
+    assert scales[0, 0] == 0x3E
+    np.testing.assert_array_equal(codes[0, :3], [0x7, 0x4, 0xC])
+    assert np.all(codes[0, 3:] == 0)
+
+
 def test_special_groups():
     v = np.zeros((1, 32), np.float32)
     v[0, 16:] = np.float32(1e-6)                   # amax/6 below half the smallest subnormal

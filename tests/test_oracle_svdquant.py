@@ -163,6 +163,17 @@ def test_prop41_bound_holds(cfg):
     assert K % 64 == 0
 
 
+def test_prop41_bound_worked_example():
+    """Prop. 4.1's right side on 1 x 2 matrices with round norms: ||X|| = 5,
+    ||X - Q(X)|| = 4, ||W|| = 2, ||W - Q(W)|| = 1, so the bound is
+    5 * 1 + 4 * (2 + 1) = 17; the product error |X W^T - Q(X) Q(W)^T| = 8 sits
+    under it."""
+    X, QX = np.array([[3.0, 4.0]]), np.array([[3.0, 0.0]])
+    W, QW = np.array([[0.0, 2.0]]), np.array([[0.0, 1.0]])
+    assert S.prop41_bound(X, W, QX, QW) == 17.0
+    assert abs((X @ W.T - QX @ QW.T)[0, 0]) == 8.0
+
+
 def test_method_beats_smoothing_beats_naive():
     t = _tiny()
     K = t.case.K
@@ -212,6 +223,20 @@ def test_refinement_keeps_the_best_split_and_one_iteration_is_plain():
     W_hat = S.smooth_weight(t.W, ref.inv_lam)
     low = (ref.L1p / ref.inv_lam.astype(np.float64)[:, None]) @ ref.L2b
     np.testing.assert_allclose(low.T + ref.R.astype(np.float64), W_hat, rtol=0, atol=1e-6)
+
+
+def test_refinement_keeps_the_best_when_a_later_split_is_worse():
+    """The iteration is not monotone: on this heavy-tailed weight (Gaussian
+    cubed, rank 6, 8 iterations) the seventh split has the smallest residual
+    quantization error and the eighth is worse, so keeping the best split and
+    keeping the last one differ."""
+    W = (np.random.default_rng(8).normal(0, 1, (32, 64)) ** 3).astype(np.float32)
+    prep = S.prepare(W, np.ones(64, np.float32), None, 6, iters=8)
+    errs = prep.refine_errors
+    best = int(np.argmin(errs))
+    assert best < len(errs) - 1 and errs[-1] > errs[best]
+    kept = np.linalg.norm(prep.R.astype(np.float64) - S.fake_quantize_weights(prep.R))
+    assert kept == pytest.approx(errs[best], rel=1e-12)
 
 
 def test_refinement_of_an_exactly_low_rank_weight_stays_put():
