@@ -37,6 +37,8 @@ MUTANTS = [
      [("np.where(neg & (mag_code != 0), mag_code | 0x8, mag_code)", "np.where(neg, mag_code | 0x8, mag_code)")], FMT),
     ("bf16_truncates", "formats.py", [("((u + 0x7FFF + lsb) >> 16)", "(u >> 16)")], FMT),
     ("bf16_ties_up", "formats.py", [("((u + 0x7FFF + lsb) >> 16)", "((u + 0x8000) >> 16)")], FMT),
+    ("e4m3_nan_as_480", "formats.py", [("mag = np.where((e == 15) & (m == 7), np.nan, mag)", "mag = mag")], FMT),
+    ("e2m1_exponent_bias_2", "formats.py", [("np.exp2(e - 1.0)", "np.exp2(e - 2.0)")], FMT),
     # NVFP4 group codec and scale layout
     ("codec_qmax_7", "codec.py", [("QMAX = 6.0", "QMAX = 7.0")], COD),
     ("codec_scale_by_reciprocal", "codec.py",
@@ -58,6 +60,16 @@ MUTANTS = [
     ("smoothing_inverted", "svdquant.py",
      [("ax[ok] ** alpha / wx[ok] ** (1.0 - alpha)", "wx[ok] ** (1.0 - alpha) / ax[ok] ** alpha")], SVD),
     ("smoothing_zero_weight_channel", "svdquant.py", [("ok = (ax > 0) & (wx > 0)", "ok = (ax > 0)")], SVD),
+    ("inv_lam_from_the_f64_lambda", "svdquant.py",
+     [("inv32 = (1.0 / lam32.astype(np.float64)).astype(np.float32)", "inv32 = (1.0 / lam).astype(np.float32)")], SVD),
+    ("l1_rounded_before_the_fold", "svdquant.py", [("round_bf16(L1 * inv64)", "round_bf16(L1) * inv64")], SVD),
+    ("l2_not_rounded", "svdquant.py", [("round_bf16(L1 * inv64), round_bf16(L2)", "round_bf16(L1 * inv64), L2")], SVD),
+    ("activations_not_smoothed", "svdquant.py",
+     [("return quantize_groups(smooth_activations(X, inv_lam))", "return quantize_groups(np.asarray(X, np.float32))")],
+     SVD),
+    ("lora_on_smoothed_x", "svdquant.py",
+     [("L1p = np.concatenate([prep.L1p, A], axis=1)",
+       "L1p = np.concatenate([prep.L1p, A * prep.inv_lam.astype(np.float64)[:, None]], axis=1)")], SVD),
     ("svd_sigma_dropped", "svdquant.py", [("L1 = vt[:r].T * s[:r][None, :]", "L1 = vt[:r].T")], SVD),
     ("residual_sign", "svdquant.py", [("R = (W_hat - low.T)", "R = (W_hat + low.T)")], SVD),
     ("residual_ignores_smoothing", "svdquant.py",
@@ -94,7 +106,12 @@ MUTANTS = [
        "                (c[..., 2 * k + 1].astype(np.uint64) << np.uint64(16 + 4 * k))",
        "word |= (c[..., 2 * k].astype(np.uint64) << np.uint64(8 * k)) | \\\n"
        "                (c[..., 2 * k + 1].astype(np.uint64) << np.uint64(8 * k + 4))")], I4),
+    ("int4_no_sign_extension", "int4.py", [("return np.where(out >= 8, out - 16, out).astype(np.int8)",
+                                            "return out.astype(np.int8)")], I4),
     # LayerNorm front end
+    ("norm_steps_in_float64", "norm.py",
+     [("d = (Z - mu).astype(np.float32)\n    n = (d * rstd).astype(np.float32)",
+       "d = Z.astype(np.float64) - mu\n    n = d * rstd")], NRM),
     ("norm_eps_dropped", "norm.py", [("1.0 / np.sqrt(var + eps)", "1.0 / np.sqrt(var)")], NRM),
     ("norm_sample_variance", "norm.py",
      [("var = ((Z - mu[:, None]) ** 2).mean(axis=1)", "var = ((Z - mu[:, None]) ** 2).sum(axis=1) / (Z.shape[1] - 1)")],

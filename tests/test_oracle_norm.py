@@ -37,3 +37,19 @@ def test_normalized_rows_have_zero_mean_unit_variance():
     np.testing.assert_allclose(x.mean(axis=1), 0.0, atol=2e-3)
     np.testing.assert_allclose(x.var(axis=1), 1.0, rtol=5e-3)
     np.testing.assert_array_equal(x, round_bf16(x))       # bf16 values
+
+
+def test_normalize_rounds_each_step_in_fp32():
+    """Each of the four steps rounds to fp32 before the last rounding to bf16.
+    Worked element (fp32 bit patterns): z = 0x4067A449 (3.6194022),
+    mu = 0xBF156111 (-0.58351237), rstd = 0x3F8D8666, a = 0x3F84A6F0,
+    c = 0x3C4837D2.  The fp32 steps give z - mu = 4.2029147 (the exact
+    difference 4.2029145 rounds up), times rstd 4.6470118, times a 4.815905,
+    plus c 4.8281255: above the midpoint 4.828125 of the bf16 values 4.8125
+    and 4.84375, so x = 4.84375.  Kept in float64 until the product with a,
+    the same element gives 4.8159046 + c = 4.828125, the midpoint itself,
+    which ties to the even 4.8125."""
+    bits = np.array([0x4067A449, 0xBF156111, 0x3F8D8666, 0x3F84A6F0, 0x3C4837D2], np.uint32)
+    z, mu, rstd, a, c = bits.view(np.float32)
+    x = ON.normalize(np.array([[z]]), np.array([mu]), np.array([rstd]), np.array([a]), np.array([c]))
+    assert x[0, 0] == np.float32(4.84375)

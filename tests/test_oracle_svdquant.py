@@ -45,6 +45,17 @@ def test_smoothing_hand_example():
     assert lam[0] == np.float32(8 ** 0.25 / 2 ** 0.75)
 
 
+def test_inverse_smoothing_is_the_reciprocal_of_the_stored_lambda():
+    """inv_lam is fp32(1 / lam) of the fp32 lam the layer keeps.  Activation
+    maximum 1, weight maximum 3: lam = 1/sqrt(3) rounds to fp32 0.57735026
+    (0x3F13CD3A, 1.0e-8 low), whose reciprocal sqrt(3) (1 + 1.8e-8) rounds to
+    1.7320509 (0x3FDDB3D8), one ulp above fp32(sqrt(3)) (0x3FDDB3D7), which
+    the reciprocal of the unrounded lam would give."""
+    lam, inv = S.smoothing_factors(np.array([1.0], np.float32), np.array([[3.0]], np.float32))
+    assert lam.view(np.uint32)[0] == 0x3F13CD3A
+    assert inv.view(np.uint32)[0] == 0x3FDDB3D8
+
+
 def test_smoothing_preserves_product():
     t = _tiny()
     lam, inv = S.smoothing_factors(t.act_absmax, t.W)
