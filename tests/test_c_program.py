@@ -1,0 +1,57 @@
+"""The boundary from C: include/svdq.h compiles as strict C99 (no C++ types in
+any signature) and a C program linked against the library runs its host-only
+entry points and the host-side argument checks, with no GPU."""
+
+import os
+import shutil
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+LIBDIR = os.path.join(ROOT, "rank_outlier_gemm_b200")
+
+C_SRC = r"""
+#include <stdio.h>
+#include <string.h>
+#include "svdq.h"
+
+int main(void) {
+  svdq_prepare_opts o;
+  svdq_prepare_opts_default(&o);
+  if (o.rank != 32 || o.alpha != 0.5f || o.format != SVDQ_FORMAT_NVFP4) return 10;
+  if (svdq_act_codes_bytes(7, 128) != 7 * 64) return 11;
+  if (svdq_act_sf_bytes(129, 64) != 256 * 4) return 12;
+  if (strstr(svdq_version(), "sm_100a") == NULL) return 13;
+
+  /* K = 96 is not a multiple of 64: rejected on the host, no handle made */
+  static uint16_t W[32 * 96];
+  float amax[96];
+  for (int i = 0; i < 96; ++i) amax[i] = 1.0f;
+  svdq_weights* w = NULL;
+  svdq_status st = svdq_prepare_weights(W, amax, NULL, 32, 96, &o, NULL, &w);
+  if (st != SVDQ_ERR_INVALID_ARG || w != NULL) return 20;
+  if (strstr(svdq_last_error(), "multiple of 64") == NULL) return 21;
+
+  /* a null weights handle is an invalid argument for every runtime call */
+  st = svdq_linear_w4a4(NULL, NULL, NULL, NULL, 1, NULL, NULL);
+  if (st != SVDQ_ERR_INVALID_ARG) return 30;
+  printf("ok %s\n", svdq_version());
+  return 0;
+}
+"""
+
+
+@pytest.mark.skipif(shutil.which("gcc") is None, reason="no C compiler")
+def test_header_is_c99_and_a_c_program_links_and_runs(tmp_path):
+    lib = os.path.join(LIBDIR, "libsvdq.so")
+    assert os.path.exists(lib), "build the library first (__graft_entry__.build())"
+    src = tmp_path / "abi.c"
+    src.write_text(C_SRC)
+    exe = tmp_path / "abi"
+    subprocess.run(["gcc", "-std=c99", "-pedantic", "-Wall", "-Wextra", "-Werror", f"-I{ROOT}/include",
+                    str(src), "-o", str(exe), f"-L{LIBDIR}", "-lsvdq", f"-Wl,-rpath,{LIBDIR}"],
+                   check=True, capture_output=True, text=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
+    assert r.stdout.startswith("ok ")
