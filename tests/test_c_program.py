@@ -33,9 +33,41 @@ int main(void) {
   if (st != SVDQ_ERR_INVALID_ARG || w != NULL) return 20;
   if (strstr(svdq_last_error(), "multiple of 64") == NULL) return 21;
 
-  /* a null weights handle is an invalid argument for every runtime call */
-  st = svdq_linear_w4a4(NULL, NULL, NULL, NULL, 1, NULL, NULL);
-  if (st != SVDQ_ERR_INVALID_ARG) return 30;
+  /* a null weights handle is an invalid argument for every call that takes one
+     (sizes: 0), and the check comes before any GPU work */
+  const svdq_weights* nw = NULL;
+  double errs[4];
+  int n = 0, k = 0, r = 0, rp = 0, fmt = 0;
+  float aw = 0.0f;
+  svdq_status got[] = {
+      svdq_linear_w4a4(nw, NULL, NULL, NULL, 1, NULL, NULL),
+      svdq_weights_refine_errors(nw, errs, 4, &n),
+      svdq_weights_format(nw, &fmt),
+      svdq_attach_lora(NULL, NULL, NULL, 16, 1.0f, NULL),
+      svdq_quantize_act_lowrank_down(nw, NULL, 1, NULL, NULL, NULL, NULL),
+      svdq_norm_quantize_act_lowrank_down(nw, NULL, 1, NULL, NULL, NULL, NULL, NULL, NULL, NULL),
+      svdq_forward_norm(nw, NULL, 1, NULL, NULL, 1e-6f, NULL, NULL, 0, NULL),
+      svdq_forward(nw, NULL, 1, NULL, NULL, 0, NULL),
+      svdq_forward_host(nw, NULL, 1, NULL, NULL, 0, NULL),
+      svdq_forward_noalloc(nw, NULL, 1, NULL, NULL),
+      svdq_weights_info(nw, &n, &k, &r, &rp, &aw),
+      svdq_weights_export(nw, NULL, NULL, NULL, NULL, NULL, NULL, NULL),
+      svdq_debug_launch_stalled_act(nw, NULL, 1, NULL, NULL, NULL, NULL),
+      svdq_debug_linear_w4a4_ksplit(nw, NULL, NULL, NULL, 1, NULL, 2, NULL),
+      svdq_act_row_stats(NULL, 1, 64, 1e-6f, NULL, NULL),
+      svdq_search_alpha(NULL, NULL, 1, NULL, 16, 64, NULL, 0, &o, NULL, errs, &n),
+      svdq_selftest_codec(NULL),
+  };
+  for (unsigned i = 0; i < sizeof(got) / sizeof(got[0]); ++i)
+    if (got[i] != SVDQ_ERR_INVALID_ARG) {
+      printf("call %u returned %d\n", i, (int)got[i]);
+      return 30;
+    }
+  if (svdq_weights_sf_bytes(nw) != 0 || svdq_lowrank_bytes(nw, 8) != 0 ||
+      svdq_forward_workspace_bytes(nw, 8) != 0 || svdq_forward_norm_workspace_bytes(nw, 8) != 0 ||
+      svdq_forward_host_workspace_bytes(nw, 8) != 0)
+    return 31;
+  if (svdq_weights_destroy(NULL) != SVDQ_OK) return 32;
   printf("ok %s\n", svdq_version());
   return 0;
 }
