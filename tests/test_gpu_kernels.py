@@ -301,6 +301,39 @@ def test_output_only_16_byte_aligned():
     assert torch.isnan(buf[:8].float()).all() and torch.isnan(buf[8 + M * N:].float()).all()
 
 
+def test_staged_store_clips_a_ragged_row_block():
+    """The GEMM epilogue's staged TMA stores (tiles of >= 8 K steps that are not
+    their CTA's last) on a row block that ends inside a warp's 32-row box:
+    M = 3900, so the last block holds rows 3840-3899 and its second warp's box
+    is 28 rows of Y and 4 past it; K = 2048 at rank 0 (8 K steps); 31 x 8 = 248
+    tiles, so CTAs 0-99 take two and the ragged block's tiles 30, 61 and 92 go
+    through the staged path.  Y matches the oracle on rows around the ragged
+    block, every element of Y is written, and guard rows after Y keep their NaNs."""
+    L = G.lib()
+    M, K, N = 3900, 2048, 2048
+    rng = np.random.default_rng(3900)
+    X = rng.normal(0, 1, (M, K)).astype(np.float32)
+    X[:, rng.choice(K, 10, replace=False)] *= 30
+    Xb = f32_to_bf16_bits(X)
+    Xf = OF.bf16_bits_to_f64(Xb).astype(np.float32)
+    W = rng.normal(0, 0.02, (N, K)).astype(np.float32)
+    bias = rng.normal(0, 0.01, N).astype(np.float32)
+    _, inv_lam = OS.smoothing_factors(np.abs(Xf).max(axis=0), W)
+    prep = _rank0_prep(W, inv_lam, bias)
+    w = G.weights_from_oracle(prep)
+    _, xq, xsf, T = G.run_act(w, Xb)
+    guard = 64
+    buf = torch.full(((M + guard) * N,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    Y = buf[:M * N].view(M, N)
+    L.svdq_linear_w4a4(w, xq, xsf, T, M, Y)
+    assert L.svdq_check_device_errors() == 0
+    assert torch.isnan(buf[M * N:].float()).all()
+    Yh = Y.float().cpu().numpy().astype(np.float64)
+    assert np.all(np.isfinite(Yh))
+    rows = np.r_[0:16, 3830:3900]
+    G.check_Y(Yh[rows], OS.linear(prep, Xf, rows=rows))
+
+
 def test_library_prepare_invariants():
     """The library's own host SVD split: inv_lam as the oracle's, L1 L2 + R
     reconstructs W_hat, and the split is near the Eckart-Young optimum."""
