@@ -381,7 +381,7 @@ def _cublaslt_fp4_us(torch, M, K, N, dev, stream, reps):
     try:
         return 1e3 * _time_ms(torch, stream, lambda: torch._scaled_mm(a, b.t(), sa, sb, out_dtype=torch.bfloat16),
                               reps)
-    except (RuntimeError, TypeError) as ex:  # no NVFP4 kernel in this build
+    except (RuntimeError, TypeError) as ex:  # this torch has no NVFP4 kernel
         print(f"cuBLASLt NVFP4 GEMM unavailable: {str(ex)[:200]}", file=sys.stderr)
         return None
 

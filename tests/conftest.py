@@ -15,7 +15,7 @@ def pytest_configure(config):
 
 def pytest_collection_modifyitems(config, items):
     # GPU tests are skipped (not failed) when no GPU is visible; `-m gpu` on a
-    # GPU machine runs them.  A GPU machine without the built library fails loudly.
+    # machine with a B200 runs them; there, a missing built library fails loudly.
     try:
         import torch
         has_gpu = torch.cuda.is_available()
