@@ -359,6 +359,37 @@ def test_library_prepare_invariants():
     assert e_lib < 1.5 * e_orc + 1e-3
 
 
+@pytest.mark.parametrize("name", ["attn_out", "qkv", "mlp_up", "mlp_down"])
+def test_bench_configuration_full_size_sampled(name):
+    """The FLUX.1 double-block layers exactly as the benchmark times them: full
+    M = 4608, weights prepared by the library's own host SVD at rank 32, both
+    kernels.  The oracle evaluates the library's exported split on 96 rows x
+    256 columns spread over the output: the weight codes and scales of those
+    columns and the activation codes and scales of those rows are bit-exact,
+    and Y there is within the layer tolerance."""
+    L = G.lib()
+    case = [c for c in config_cases("flux") if c.name == name][0]
+    t = make_layer_inputs(case)
+    w = L.svdq_prepare_weights(t.W_bits, t.act_absmax, t.bias_bits, rank=case.rank, keep_residual=True)
+    ex = L.svdq_weights_export(w, residual=True)
+    Y, (xq, xsf, T) = G.run_layer(w, t.X_bits)
+    M, N = Y.shape
+    rows = np.r_[0:32, M // 2:M // 2 + 32, M - 32:M]
+    cols = np.r_[0:64, N // 2 - 64:N // 2 + 64, N - 64:N]
+    inv = ex["inv_lam"]
+    Rp = ex["residual"][cols]
+    codes, scales = OC.quantize_groups(Rp)
+    np.testing.assert_array_equal(ex["codes"][cols], OC.pack_codes(codes))
+    np.testing.assert_array_equal(OC.atoms_to_scales(ex["sf"], N, case.K // 16)[cols], scales)
+    prep = OS.Prepared(len(cols), case.K, ex["rank"], (1.0 / inv.astype(np.float64)).astype(np.float32), inv,
+                       OF.bf16_bits_to_f64(ex["L1p"]), OF.bf16_bits_to_f64(ex["L2"])[:, cols],
+                       (Rp.astype(np.float64) * ex["alpha_w"]).astype(np.float32), ex["alpha_w"], Rp, codes, scales,
+                       ex["bias"][cols].astype(np.float64))
+    G.check_codes(xq, xsf, t.X, inv, rows=rows)
+    G.check_T(T, t.X, prep, rows=rows)
+    G.check_Y(Y[np.ix_(rows, cols)], OS.linear(prep, t.X, rows=rows))
+
+
 def test_library_refinement_matches_oracle():
     """Refined split (SVDQuant §4.2; the update rule is a reading of its iterations):
     the library's residual quantization errors follow the oracle's (exact SVD)
