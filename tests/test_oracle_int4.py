@@ -135,6 +135,25 @@ def test_layer_low_rank_and_bias_terms():
     np.testing.assert_allclose(y - main, OS.lowrank_down(X, prep.base) @ prep.L2b + b, rtol=0, atol=1e-12)
 
 
+def test_lora_on_the_int4_layer():
+    """A LoRA attached to the INT4 layer (SVDQuant §2, §5.2: absorbed into the
+    low-rank branch without re-quantizing R) adds scale (X A) B to the output
+    and leaves the residual's codes and scales as they were."""
+    rng = np.random.default_rng(17)
+    K, N, r, rl = 128, 32, 8, 4
+    W = (rng.standard_normal((N, K)) * 0.05).astype(np.float32)
+    X = rng.standard_normal((6, K)).astype(np.float32)
+    A = (rng.standard_normal((K, rl)) * 0.1).astype(np.float32)
+    B = (rng.standard_normal((rl, N)) * 0.1).astype(np.float32)
+    prep = OI.prepare(W, np.abs(X).max(0), None, r)
+    withl = OI.attach_lora(prep, A, B, scale=0.5)
+    np.testing.assert_array_equal(withl.w_codes, prep.w_codes)
+    np.testing.assert_array_equal(withl.w_scales, prep.w_scales)
+    assert withl.rank == r + rl
+    added = 0.5 * (X.astype(np.float64) @ A.astype(np.float64)) @ B.astype(np.float64)
+    np.testing.assert_allclose(OI.linear(withl, X) - OI.linear(prep, X), added, rtol=0, atol=1e-12)
+
+
 def test_prop41_bound_holds_for_int4():
     rng = np.random.default_rng(13)
     X = rng.standard_normal((16, 256)).astype(np.float32)

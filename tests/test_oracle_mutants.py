@@ -90,6 +90,16 @@ MUTANTS = [
      [("round_bf16(scale * B)", "round_bf16(B)"), ("scale * B], axis=0)", "B], axis=0)")], SVD),
     ("lora_reference_uses_rounded_factor", "svdquant.py",
      [("L2 = prep.L2b if prep.lora_B_exact is None else prep.lora_B_exact", "L2 = prep.L2b")], SVD),
+    ("smooth_weight_multiplies", "svdquant.py",
+     [("return np.asarray(W, np.float64) / np.asarray(inv_lam, np.float64)[None, :]",
+       "return np.asarray(W, np.float64) * np.asarray(inv_lam, np.float64)[None, :]")], SVD),
+    ("residual_not_divided_by_alpha_w", "svdquant.py",
+     [("Rp = (R.astype(np.float64) / aw).astype(np.float32)  # exact: power of two",
+       "Rp = R.astype(np.float32)")], SVD),
+    ("fake_quantize_drops_alpha_w", "svdquant.py",
+     [("return dequantize_groups(codes, scales) * aw", "return dequantize_groups(codes, scales)")], SVD),
+    ("alpha_search_picks_the_worst", "svdquant.py",
+     [("return errs, int(np.argmin(errs))", "return errs, int(np.argmax(errs))")], SVD),
     ("refinement_keeps_last", "svdquant.py",
      [("if best is None or errors[-1] < min(errors[:-1]):", "if True:")], SVD),
     ("refinement_repeats_the_split", "svdquant.py", [("        A = W_hat - Q\n", "        A = W_hat - prep.R\n")], SVD),
@@ -108,7 +118,15 @@ MUTANTS = [
        "                (c[..., 2 * k + 1].astype(np.uint64) << np.uint64(8 * k + 4))")], I4),
     ("int4_no_sign_extension", "int4.py", [("return np.where(out >= 8, out - 16, out).astype(np.int8)",
                                             "return out.astype(np.int8)")], I4),
+    ("int4_linear_drops_lowrank", "int4.py",
+     [("return main + S.lowrank_down(X, b) @ L2[:, c] + b.bias[None, c]", "return main + b.bias[None, c]")], I4),
+    ("int4_dequant_ignores_scale", "int4.py",
+     [("return (codes.reshape(R, K // GROUP, GROUP) * s[..., None]).reshape(R, K)",
+       "return codes.reshape(R, K).astype(np.float64)")], I4),
+    ("int4_lora_dropped", "int4.py",
+     [("return dataclasses.replace(prep, base=S.attach_lora(prep.base, A, B, scale))", "return prep")], I4),
     # LayerNorm front end
+    ("norm_mean_over_tokens", "norm.py", [("mu = Z.mean(axis=1)", "mu = Z.mean(axis=1) * 0.0 + Z.mean()")], NRM),
     ("norm_steps_in_float64", "norm.py",
      [("d = (Z - mu).astype(np.float32)\n    n = (d * rstd).astype(np.float32)",
        "d = Z.astype(np.float64) - mu\n    n = d * rstd")], NRM),
