@@ -2,6 +2,7 @@
 any signature) and a C program linked against the library runs its host-only
 entry points and the host-side argument checks, with no GPU."""
 
+import ctypes
 import os
 import shutil
 import subprocess
@@ -12,6 +13,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 LIBDIR = os.path.join(ROOT, "rank_outlier_gemm_b200")
 
 C_SRC = r"""
+#include <stddef.h>
 #include <stdio.h>
 #include <string.h>
 #include "svdq.h"
@@ -68,6 +70,11 @@ int main(void) {
       svdq_forward_host_workspace_bytes(nw, 8) != 0)
     return 31;
   if (svdq_weights_destroy(NULL) != SVDQ_OK) return 32;
+  printf("layout %zu %zu %zu %zu %zu %zu %zu %zu %zu\n", sizeof(svdq_prepare_opts),
+         offsetof(svdq_prepare_opts, alpha), offsetof(svdq_prepare_opts, rank),
+         offsetof(svdq_prepare_opts, power_iters), offsetof(svdq_prepare_opts, oversample),
+         offsetof(svdq_prepare_opts, seed), offsetof(svdq_prepare_opts, keep_residual),
+         offsetof(svdq_prepare_opts, refine_iters), offsetof(svdq_prepare_opts, format));
   printf("ok %s\n", svdq_version());
   return 0;
 }
@@ -86,4 +93,12 @@ def test_header_is_c99_and_a_c_program_links_and_runs(tmp_path):
                    check=True, capture_output=True, text=True)
     r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
     assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
-    assert r.stdout.startswith("ok ")
+    layout, ok = r.stdout.splitlines()
+    assert ok.startswith("ok ")
+    # the Python binding's copy of svdq_prepare_opts has the C layout
+    from rank_outlier_gemm_b200.binding import PrepareOpts
+    P = PrepareOpts
+    want = [ctypes.sizeof(P)] + [getattr(P, f).offset for f in
+                                 ["alpha", "rank", "power_iters", "oversample", "seed", "keep_residual",
+                                  "refine_iters", "format"]]
+    assert [int(v) for v in layout.split()[1:]] == want
