@@ -80,3 +80,33 @@ def test_invalid_arguments_rejected_before_gpu():
     with pytest.raises(B.SvdqError) as e:
         B.svdq_weights_from_factors(32, 64, 0, np.ones(64, np.float32), None, None, R)
     assert e.value.status == 1
+
+
+def _prototypes():
+    """name -> (return type, parameter count) of every function the header declares."""
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    out = {}
+    for m in re.finditer(r"([A-Za-z_][\w\s\*]*?)\b(svdq_[a-z0-9_]+)\s*\(([^)]*)\)\s*;", text):
+        ret = " ".join(m.group(1).split())
+        params = m.group(3).strip()
+        n = 0 if params in ("", "void") else len(params.split(","))
+        out[m.group(2)] = (ret, n)
+    return out
+
+
+def test_binding_signatures_match_the_header():
+    """Every ctypes signature of the binding has the header's parameter count and
+    a return type of the matching kind (status and int -> c_int, size_t ->
+    c_size_t, const char* -> c_char_p, void -> None)."""
+    import ctypes
+    from rank_outlier_gemm_b200 import binding as B
+    protos = _prototypes()
+    assert set(protos) == set(B._SIGS)
+    kinds = {"svdq_status": ctypes.c_int, "int": ctypes.c_int, "size_t": ctypes.c_size_t,
+             "const char*": ctypes.c_char_p, "const char *": ctypes.c_char_p, "void": None}
+    for name, (ret, n) in protos.items():
+        res, args = B._SIGS[name]
+        assert len(args) == n, (name, len(args), n)
+        assert kinds[ret] is res, (name, ret, res)
+
