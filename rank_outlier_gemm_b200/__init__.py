@@ -11,6 +11,8 @@ import importlib
 
 
 def __getattr__(name):
+    if name == "build":  # the build script never needs the built library
+        return importlib.import_module(".build", __name__)
     binding = importlib.import_module(".binding", __name__)
     try:
         return getattr(binding, name)

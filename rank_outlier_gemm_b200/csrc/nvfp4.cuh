@@ -10,9 +10,11 @@
 // division and the reciprocal are computed by exact shortcuts, both checked
 // against the IEEE intrinsics over their whole domains by svdq_selftest_codec:
 // - amax / 6: q0 = RN(amax * RN(1/6)), then one fused correction with the
-//   exact remainder fma(-q0, 6, amax) (the classical correction step for
-//   division by a constant known in advance); for every fp32 mantissa it gives
-//   RN(amax / 6), and below the normal range the E4M3 scale is 0 either way.
+//   exact remainder fma(-q0, 6, amax), the method of Brisebarre, Muller and
+//   Raina, "Accelerating correctly rounded floating-point division when the
+//   divisor is known in advance" (IEEE Trans. Computers 53(8), 2004); for every
+//   fp32 mantissa it gives RN(amax / 6) (checked exhaustively), and below the
+//   normal range the E4M3 scale is 0 either way.
 // - 1 / decode(s): decode(s) is (1 + m/8) 2^(e-7), or m 2^-9 when e = 0, with a
 //   3-bit m, and
 //   RN(1 / (2^k x)) = 2^-k RN(1 / x) in the normal range, so a 16-entry table of
@@ -30,7 +32,9 @@ struct Fp4Group {
   uint32_t scale;   // E4M3 byte
 };
 
-// RN(x / 6) for every finite fp32 x whose quotient is normal.
+// RN(x / 6) for every finite fp32 x whose quotient is normal (Brisebarre,
+// Muller and Raina 2004: multiply by the rounded reciprocal, then one fused
+// correction with the exact remainder).
 __device__ __forceinline__ float div6_rn(float x) {
   const float c = __uint_as_float(0x3E2AAAABu);  // RN(1/6)
   const float q0 = __fmul_rn(x, c);
