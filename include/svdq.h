@@ -26,10 +26,10 @@
  *    buffers alive until the work queued on the stream has finished.  The
  *    library owns the svdq_weights handle and the device memory inside it;
  *    svdq_weights_destroy frees both.
- *  - CUDA graphs: the runtime calls (both kernels, svdq_forward and its
- *    allocation-free variant) can be captured into a graph once the same call
- *    has run eagerly on the device, since a first call sets up per-device
- *    state (error word, kernel attributes, occupancy queries).
+ *  - CUDA graphs: the runtime calls (both kernels and svdq_forward) can be
+ *    captured into a graph once the same call has run eagerly on the device,
+ *    since a first call sets up per-device state (error word, kernel
+ *    attributes, occupancy queries).
  *  - Streams: `stream` is a cudaStream_t passed as void* (NULL = the legacy
  *    default stream).  Runtime calls only enqueue work; they do not
  *    synchronize.  Weight preparation and LoRA attachment synchronize.
@@ -293,25 +293,30 @@ svdq_status svdq_forward_host(const svdq_weights* w, const void* X_host, int M, 
                               void* workspace, size_t workspace_bytes, void* stream);
 
 /*
- * svdq_forward without a workspace, for callers that must not allocate device
- * memory: code running inside a caching allocator's callbacks, a CUDA graph
- * capture whose pool forbids new allocations, or a serving loop whose memory
- * is fully reserved up front.  (The paper has no counterpart; this is a
- * deployment convenience of this library.)
+ * svdq_forward without a workspace, for callers that cannot call cudaMalloc:
+ * code running inside a caching allocator's callbacks (an allocation there
+ * re-enters the allocator or fails against its reserve), or a serving loop
+ * whose device memory is fully reserved up front.  (The paper has no
+ * counterpart; this is a deployment convenience of this library.)
  *
  * The intermediates (activation codes, scales, T) live in one static block of
- * device memory of at most 32 MiB that every GPU loading the library's device
- * code keeps until the process exits; layers whose intermediates exceed it
+ * device memory of 32 MiB per device; layers whose intermediates exceed it
  * (M*K/2 + ceil(M/128)*128*K/16 + 4*M*r_pad bytes, each rounded up to 256)
- * are rejected with SVDQ_ERR_INVALID_ARG.  The call allocates nothing: the
- * first call on a device looks up the block's device address (with that
- * device current), so make that first call before any stream capture.
+ * are rejected with SVDQ_ERR_INVALID_ARG before any GPU work.  The block is
+ * part of the library's device code: the FIRST call on a device, with that
+ * device current, looks up its device address, which makes CUDA load that
+ * code and commit the 32 MiB on the device (kept until the process exits).
+ * Make that first call before reserving the rest of the device's memory and
+ * before any stream capture.  Later calls allocate nothing: no cudaMalloc,
+ * cudaFree or allocating library routine.
  *
  * All calls on a device share the one block and leave their intermediates in
  * it; calls whose kernels overlap on the GPU (other streams, other threads)
  * race on it and must be serialized by the caller.  Nothing in the block needs
  * to start at zero.  A device-side wait that runs out is recorded in a static
- * word that this path does not report; its outputs are then unspecified.
+ * error word of this path, which svdq_check_device_errors reads and clears
+ * together with the library's other word; the outputs of that call are then
+ * unspecified.
  *   X_bf16  device, M x K bf16          Y_bf16  device, M x N bf16
  */
 svdq_status svdq_forward_noalloc(const svdq_weights* w, const void* X_bf16, int M, void* Y_bf16,
@@ -325,6 +330,10 @@ size_t svdq_forward_workspace_bytes(const svdq_weights* w, int M);
 size_t svdq_forward_host_workspace_bytes(const svdq_weights* w, int M);
 size_t svdq_forward_norm_workspace_bytes(const svdq_weights* w, int M);
 size_t svdq_weights_sf_bytes(const svdq_weights* w);       /* the handle's weight scales */
+
+/* Rank of the handle's 16-bit branch (§4.2, rank r of L1 and L2, plus the
+ * ranks of the LoRAs attached by svdq_attach_lora, §5.2); -1 for NULL. */
+int svdq_weights_rank(const svdq_weights* w);
 
 /* Shape of a handle: rank counts the SVD rank plus attached LoRA ranks, r_pad
  * is that rounded up to a multiple of 16 (the width of T's hi and lo parts). */
@@ -359,7 +368,8 @@ void svdq_set_wait_limit_ns(uint64_t ns);
 
 /*
  * Synchronizes `stream`, then reads and clears the current device's error
- * word: SVDQ_OK, SVDQ_ERR_TIMEOUT or SVDQ_ERR_DEVICE_CHECK.
+ * words (the library's, and the allocation-free path's once that path has run
+ * on the device): SVDQ_OK, SVDQ_ERR_TIMEOUT or SVDQ_ERR_DEVICE_CHECK.
  */
 svdq_status svdq_check_device_errors(void* stream);
 

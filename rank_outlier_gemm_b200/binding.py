@@ -62,6 +62,7 @@ _SIGS = {
     "svdq_lowrank_bytes": (_sz, [_vp, _i]),
     "svdq_forward_workspace_bytes": (_sz, [_vp, _i]),
     "svdq_forward_host_workspace_bytes": (_sz, [_vp, _i]),
+    "svdq_weights_rank": (_i, [_vp]),
     "svdq_weights_info": (_i, [_vp, ctypes.POINTER(_i), ctypes.POINTER(_i), ctypes.POINTER(_i),
                                ctypes.POINTER(_i), ctypes.POINTER(_f)]),
     "svdq_weights_export": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
@@ -151,7 +152,8 @@ class Weights:
                 "format": {v: k for k, v in FORMATS.items()}[fmt.value]}
 
     def __del__(self):
-        if getattr(self, "handle", None):
+        # at interpreter exit the module globals may already be gone
+        if getattr(self, "handle", None) and _lib is not None:
             _lib.svdq_weights_destroy(self.handle)
             self.handle = None
 
@@ -292,6 +294,10 @@ def svdq_forward_host_workspace_bytes(w: Weights, M: int) -> int:
 
 def svdq_weights_info(w: Weights) -> dict:
     return w.info
+
+
+def svdq_weights_rank(w: Weights) -> int:
+    return int(_lib.svdq_weights_rank(w.handle))
 
 
 def svdq_weights_export(w: Weights, residual: bool = False) -> dict:

@@ -651,6 +651,8 @@ svdq_status svdq_forward_host(const svdq_weights* w, const void* X_host, int M, 
   return SVDQ_OK;
 }
 
+int svdq_weights_rank(const svdq_weights* w) { return w ? w->rank : -1; }
+
 svdq_status svdq_weights_info(const svdq_weights* w, int* N, int* K, int* rank, int* r_pad, float* alpha_w) {
   if (!w) return fail(SVDQ_ERR_INVALID_ARG, "null weights handle");
   if (N) *N = w->N;
@@ -693,12 +695,20 @@ svdq_status svdq_check_device_errors(void* stream) {
   SVDQ_CUDA_TRY(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
   int* word = device_error_word();
   if (!word) return fail(SVDQ_ERR_CUDA, "device error word unavailable");
-  int v = 0;
-  SVDQ_CUDA_TRY(cudaMemcpy(&v, word, sizeof(int), cudaMemcpyDeviceToHost));
-  if (v != 0) {
-    SVDQ_CUDA_TRY(cudaMemset(word, 0, sizeof(int)));
-    return fail(static_cast<svdq_status>(v), "device error word = %d", v);
+  // the allocation-free path keeps its own static word; read and clear both
+  int* words[2] = {word, noalloc_error_word_if_ready()};
+  int first = 0;
+  for (int* wp : words) {
+    if (!wp) continue;
+    int v = 0;
+    SVDQ_CUDA_TRY(cudaMemcpy(&v, wp, sizeof(int), cudaMemcpyDeviceToHost));
+    if (v != 0) {
+      const int zero = 0;
+      SVDQ_CUDA_TRY(cudaMemcpy(wp, &zero, sizeof(int), cudaMemcpyHostToDevice));
+      if (!first) first = v;
+    }
   }
+  if (first) return fail(static_cast<svdq_status>(first), "device error word = %d", first);
   return SVDQ_OK;
 }
 

@@ -1,13 +1,16 @@
 // svdq_forward_noalloc: both kernels of the layer with their intermediates
 // (activation codes, scales and the low-rank T) in a fixed block of static
 // device memory instead of a caller-provided workspace, for callers that must
-// not allocate: code running inside a caching allocator's callbacks, a CUDA
-// graph capture that forbids new allocations, or a serving loop whose memory
-// pool is already fully reserved.
+// not allocate: code running inside a caching allocator's callbacks (a
+// cudaMalloc there can re-enter the allocator or fail against its reserve), or
+// a serving loop whose device memory is fully reserved up front.
 //
-// The block lives for as long as the library is loaded, on every GPU that
-// loads it.  In host code its name is only a host-side stand-in, so its device
-// address is looked up once per device, with that device current, and cached.
+// The block belongs to this file's device-code module.  CUDA loads a module on
+// a device the first time one of its symbols is used there, so the block is
+// committed (32 MiB) by the first svdq_forward_noalloc call on each device,
+// which looks up its device address -- in host code the array's name is only a
+// host-side stand-in -- and from then on stays until the process exits.  Every
+// later call allocates nothing.
 #include <mutex>
 
 #include "svdq_internal.h"
@@ -48,6 +51,20 @@ svdq_status scratch_for_current_device(DeviceScratch* out) {
 }
 
 }  // namespace
+
+namespace svdq {
+
+// The static error word of this path on the current device, or nullptr while
+// no svdq_forward_noalloc call has set the path up there (the lookup is not
+// made here, so reading errors never loads the block).
+int* noalloc_error_word_if_ready() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  return g_scratch[dev].err;
+}
+
+}  // namespace svdq
 
 using namespace svdq;
 

@@ -32,6 +32,9 @@ svdq_status cuda_fail(cudaError_t e, const char* what);
 
 // Device error word of the current device (lazily allocated, zeroed).
 int* device_error_word();
+// The allocation-free path's static error word on the current device, or
+// nullptr if that path has not run there yet.
+int* noalloc_error_word_if_ready();
 uint64_t wait_limit_ns();
 // SVDQ_OK if the current device is sm_100, else SVDQ_ERR_UNSUPPORTED_DEVICE.
 svdq_status check_device();

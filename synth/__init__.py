@@ -14,6 +14,7 @@ from .workloads import (  # noqa: F401
     make_layer_inputs,
     make_fp4_grid_inputs,
     make_int4_grid_inputs,
+    make_lora_factors,
     bf16_bits_to_f32,
     f32_to_bf16_bits,
 )

@@ -164,6 +164,17 @@ def make_layer_inputs(case: LayerCase, M: Optional[int] = None) -> LayerInputs:
     return out
 
 
+def make_lora_factors(K: int, N: int, r_l: int, seed: int):
+    """A LoRA of rank ``r_l`` for a K -> N layer: A (K x r_l) and B (r_l x N)
+    drawn N(0, 0.01) like the configured small-M LoRA, rounded to bf16.
+    Returns (A_bits, A, B_bits, B)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    A = rng.normal(0.0, 0.01, size=(K, r_l)).astype(np.float32)
+    B = rng.normal(0.0, 0.01, size=(r_l, N)).astype(np.float32)
+    Ab, Bb = f32_to_bf16_bits(A), f32_to_bf16_bits(B)
+    return Ab, bf16_bits_to_f32(Ab), Bb, bf16_bits_to_f32(Bb)
+
+
 # Magnitudes a 4-bit E2M1 element can take (used only to build inputs that lie
 # on the FP4 grid already).
 _FP4_GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0], dtype=np.float32)

@@ -70,6 +70,7 @@ int main(void) {
       svdq_forward_host_workspace_bytes(nw, 8) != 0)
     return 31;
   if (svdq_weights_destroy(NULL) != SVDQ_OK) return 32;
+  if (svdq_weights_rank(nw) != -1) return 33;
   printf("layout %zu %zu %zu %zu %zu %zu %zu %zu %zu\n", sizeof(svdq_prepare_opts),
          offsetof(svdq_prepare_opts, alpha), offsetof(svdq_prepare_opts, rank),
          offsetof(svdq_prepare_opts, power_iters), offsetof(svdq_prepare_opts, oversample),
