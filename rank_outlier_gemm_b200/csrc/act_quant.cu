@@ -209,6 +209,24 @@ __global__ void __launch_bounds__(kThreads, 2) act_quant_lowrank_kernel(
       const int s = i % kStages;
       const uint32_t ph = (i / kStages) & 1;
       if (!wait_warp(&sh->full[s], ph, wc)) break;
+      if (m0 + 16 * wq >= p.M) {
+        // every row of this warp is padding (the TMA filled it with zeros): no
+        // codes to write, and the scales of padding rows are 0 by definition
+        __syncwarp();
+        if (lane == 0) {
+          if (kNorm) mbar_arrive(&sh->normed[s]);
+          mbar_arrive(&sh->empty[s]);
+        }
+        const int kt = t0 + i;
+        if (h == 0) {
+          if constexpr (kInt4)
+            reinterpret_cast<uint16_t*>(p.xsf)[static_cast<size_t>(kt) * p.m_pad + m] = 0;
+          else
+            *reinterpret_cast<uint32_t*>(p.xsf + (static_cast<size_t>(mb) * p.kt_total + kt) * 512 +
+                                         (row & 31) * 16 + (row >> 5) * 4) = 0u;
+        }
+        continue;
+      }
       uint8_t* xrow = xs + s * kXTile + row * 128;
       const float4* inv4 = reinterpret_cast<const float4*>(invs + s * kAux) + 8 * h;
       if constexpr (kNorm) {

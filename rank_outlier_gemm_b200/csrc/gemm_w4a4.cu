@@ -50,7 +50,7 @@ using namespace dev;
 
 constexpr int kBN = 256;
 constexpr int kThreads = 320;
-constexpr int kStages = 4;
+constexpr int kMaxStages = 4;
 constexpr int kATile = 128 * 128;               // 128 rows x 128 bytes (256 FP4 along K)
 constexpr int kBTile = kBN * 128;               // 256 rows x 128 bytes
 constexpr int kSfa = 2048;                      // four 512-byte atoms
@@ -60,7 +60,7 @@ constexpr int kSfCols = 16 + 32;                // TMEM columns of one scale slo
 constexpr int kSfSlots = 2;                     // 2 x 48 = 96 columns
 constexpr int kMaxSplit = 8;                    // portable cluster size
 constexpr int kPartStride = kBN + 4;            // fp32 words per partial row (bank spread)
-static_assert(128 * kPartStride * 4 <= kStages * kStage, "partials fit in the stage buffers");
+static_assert(128 * kPartStride * 4 <= 3 * kStage, "partials fit in the stage buffers");
 
 struct K2Params {
   int M, N, K, r_pad;
@@ -81,10 +81,16 @@ struct K2Params {
   uint64_t wait_ns;
 };
 
+// Two configurations: 4 operand stages and one Y staging buffer per epilogue
+// warp (long K: the main loop hides the epilogue), or 3 stages and a ring of
+// 4 Y buffers per warp (short K: the epilogue is the longer of the two, and
+// its TMA stores then overlap instead of waiting for each other).
+template <int kStages, int kYBufs>
 struct K2Shared {
-  // one 32 x 32 bf16 chunk of Y per epilogue warp, in the 64-byte-swizzled
+  // per epilogue warp, kYBufs 32 x 32 bf16 chunks of Y in the 64-byte-swizzled
   // layout of the Y tensor map
-  alignas(1024) uint8_t ystage[4][2048];
+  alignas(1024) uint8_t ystage[4][kYBufs][2048];
+  float bias[kBN];  // the current tile's bias columns (fp32)
   uint64_t full[kStages];
   uint64_t empty[kStages];
   uint64_t sf_full[kSfSlots];
@@ -95,6 +101,7 @@ struct K2Shared {
   uint64_t done;
   uint32_t tmem_base;
   int abort;
+  int epi_stop;  // the epilogue warps leave their tile loop together
 };
 
 __device__ __noinline__ bool wait_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
@@ -115,11 +122,12 @@ __device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
 // in pairs.  alpha_w is a power of two, so alpha_w * acc is exact (outside the
 // subnormal range) and one fused multiply-add rounds exactly like the product
 // followed by the sum.
-__device__ __forceinline__ void epi_pack(const uint32_t (&r)[32], const K2Params& p, int n, uint32_t (&packed)[16]) {
-  const float4* b4 = reinterpret_cast<const float4*>(p.bias + n);  // padded to a multiple of 256
+__device__ __forceinline__ void epi_pack(const uint32_t (&r)[32], const K2Params& p, const float* bias_s,
+                                         uint32_t (&packed)[16]) {
+  const float4* b4 = reinterpret_cast<const float4*>(bias_s);  // this chunk's 32 bias columns (shared)
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const float4 bv = __ldg(b4 + i);
+    const float4 bv = b4[i];
     const float y0 = __fmaf_rn(__uint_as_float(r[4 * i + 0]), p.alpha_w, bv.x);
     const float y1 = __fmaf_rn(__uint_as_float(r[4 * i + 1]), p.alpha_w, bv.y);
     const float y2 = __fmaf_rn(__uint_as_float(r[4 * i + 2]), p.alpha_w, bv.z);
@@ -137,12 +145,18 @@ __device__ __forceinline__ void epi_pack(const uint32_t (&r)[32], const K2Params
 // >= M; its issue waits for the previous chunk's store to read the buffer, so a
 // chunk takes longer than a direct store: used while the next tile's main loop
 // is long enough to hide it.
+template <int kYBufs>
 __device__ __forceinline__ void store_chunk_tma(const uint32_t (&r)[32], const K2Params& p, const CUtensorMap* map_y,
-                                                uint8_t* stage, uint32_t lane, int m_warp, int n) {
+                                                uint8_t (*ys)[2048], int& ybuf, const float* bias_s, uint32_t lane,
+                                                int m_warp, int n) {
   if (m_warp >= p.M || n >= p.N) return;
   uint32_t packed[16];
-  epi_pack(r, p, n, packed);
-  if (lane == 0) bulk_wait_read<0>();  // the previous chunk's store has read the buffer
+  epi_pack(r, p, bias_s, packed);
+  // the ring's buffers are used by the warp's stores in turn: the store that
+  // last used this one is kYBufs groups back, so at most kYBufs - 1 may still read
+  uint8_t* stage = ys[ybuf];
+  ybuf = ybuf + 1 == kYBufs ? 0 : ybuf + 1;
+  if (lane == 0) bulk_wait_read<kYBufs - 1>();
   __syncwarp();
   // 64-byte rows, 64-byte swizzle: row r's 16-byte piece i sits at piece i ^ ((r >> 1) & 3)
   uint4* row = reinterpret_cast<uint4*>(stage + lane * 64);
@@ -160,10 +174,11 @@ __device__ __forceinline__ void store_chunk_tma(const uint32_t (&r)[32], const K
 
 // The same chunk stored straight from registers: each lane writes its row's 64
 // bytes as whole 32-byte sectors when Y allows it (else 16-byte halves).
-__device__ __forceinline__ void store_chunk_direct(const uint32_t (&r)[32], const K2Params& p, int m, int n) {
+__device__ __forceinline__ void store_chunk_direct(const uint32_t (&r)[32], const K2Params& p, const float* bias_s,
+                                                   int m, int n) {
   if (m >= p.M || n >= p.N) return;
   uint32_t packed[16];
-  epi_pack(r, p, n, packed);
+  epi_pack(r, p, bias_s, packed);
   uint16_t* dst = p.Y + static_cast<size_t>(m) * p.N + n;
   if (p.y32) {
 #pragma unroll
@@ -181,14 +196,15 @@ __device__ __forceinline__ void store_chunk_direct(const uint32_t (&r)[32], cons
 // One warp's share of a tile's epilogue (its 32 rows, 256 columns): chunks 0-2
 // first, whose accumulator columns then take the next tile's scale slots, then
 // chunks 3-7, each chunk's TMEM load in flight while the one before is stored.
-template <bool kTma>
+template <bool kTma, int kYBufs>
 __device__ __forceinline__ void epilogue_tile(const K2Params& p, const CUtensorMap* map_y, uint32_t acc,
-                                              uint64_t* sfreg_free, uint8_t* ys, uint32_t lane, int m_warp, int n0) {
+                                              uint64_t* sfreg_free, uint8_t (*ys)[2048], int& ybuf,
+                                              const float* bias_s, uint32_t lane, int m_warp, int n0) {
   auto put = [&](const uint32_t(&rr)[32], int c) {
     if constexpr (kTma)
-      store_chunk_tma(rr, p, map_y, ys, lane, m_warp, n0 + 32 * c);
+      store_chunk_tma<kYBufs>(rr, p, map_y, ys, ybuf, bias_s + 32 * c, lane, m_warp, n0 + 32 * c);
     else
-      store_chunk_direct(rr, p, m_warp + static_cast<int>(lane), n0 + 32 * c);
+      store_chunk_direct(rr, p, bias_s + 32 * c, m_warp + static_cast<int>(lane), n0 + 32 * c);
   };
   uint32_t r[3][32];
 #pragma unroll
@@ -246,15 +262,20 @@ __device__ __forceinline__ void split_reduce(const K2Params& p, const float* par
   }
 }
 
+// Named barrier of the four epilogue warps (ids 0 and 1 are __syncthreads and unused).
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
+
+template <int kStages, int kYBufs>
 __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
     const __grid_constant__ CUtensorMap map_xq, const __grid_constant__ CUtensorMap map_wq,
     const __grid_constant__ CUtensorMap map_t, const __grid_constant__ CUtensorMap map_l2,
     const __grid_constant__ CUtensorMap map_y,
     const K2Params p) {
+  using Shared = K2Shared<kStages, kYBufs>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  K2Shared* sh = reinterpret_cast<K2Shared*>(smem + kStages * kStage);
-  static_assert(offsetof(K2Shared, ystage) == 0, "Y staging buffers keep the 1024-byte alignment the swizzle needs");
+  Shared* sh = reinterpret_cast<Shared*>(smem + kStages * kStage);
+  static_assert(offsetof(Shared, ystage) == 0, "Y staging buffers keep the 1024-byte alignment the swizzle needs");
   static_assert((kStages * kStage) % 1024 == 0, "stage buffers keep 1024-byte alignment");
 
   const uint32_t warp = warp_id(), lane = lane_id();
@@ -287,6 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
     }
     mbar_init(&sh->done, 1);
     sh->abort = 0;
+    sh->epi_stop = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -516,17 +538,27 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
     const int q = warp & 3;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     const int row = q * 32 + lane;
-    uint8_t* ys = sh->ystage[warp - 6];
+    uint8_t(*ys)[2048] = sh->ystage[warp - 6];
+    const int et = static_cast<int>(threadIdx.x) - 6 * 32;  // 0..127 over the epilogue warps
+    int ybuf = 0;  // next buffer of the warp's Y staging ring
     int j = 0;
     for (int t = tile0; t < ntiles_total; t += tile_step, ++j) {
       const int a = j & 1;
       const int m_warp = (t % p.mtiles) * 128 + q * 32;
       const int m = m_warp + static_cast<int>(lane);
       const int n0 = (t / p.mtiles) * kBN;
-      // staged TMA stores while another tile's main loop follows; the CTA's last
-      // tile (nothing left to overlap) and short tiles store directly
-      const bool tma = p.tma_y && t + tile_step < ntiles_total;
-      if (!wait_warp(&sh->acc_full[a], (j >> 1) & 1, wc)) break;
+      // staged TMA stores while another tile's main loop follows (or always,
+      // with a ring of buffers); the CTA's last tile stores directly
+      const bool tma = p.tma_y && (kYBufs > 1 || t + tile_step < ntiles_total);
+      // this tile's bias columns (the bias is padded to a multiple of 256),
+      // loaded before the wait so that the load latency hides under the MMAs
+      const float2 bpre = __ldg(reinterpret_cast<const float2*>(p.bias + n0) + et);
+      if (!wait_warp(&sh->acc_full[a], (j >> 1) & 1, wc) && lane == 0) sh->epi_stop = 1;
+      epi_bar();  // every epilogue warp is done with the previous tile's bias
+      const bool stop = sh->epi_stop != 0;  // the same for all four warps (written before the barrier)
+      if (!stop) reinterpret_cast<float2*>(sh->bias)[et] = bpre;
+      epi_bar();
+      if (stop) break;
       tc_fence_after();
       if (S > 1) {
         // split-K (one tile per CTA): this split's partial rows into the
@@ -553,9 +585,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
         continue;
       }
       if (tma)
-        epilogue_tile<true>(p, &map_y, tmem + a * 256 + lane_off, &sh->sfreg_free[a], ys, lane, m_warp, n0);
+        epilogue_tile<true, kYBufs>(p, &map_y, tmem + a * 256 + lane_off, &sh->sfreg_free[a], ys, ybuf, sh->bias,
+                                    lane, m_warp, n0);
       else
-        epilogue_tile<false>(p, &map_y, tmem + a * 256 + lane_off, &sh->sfreg_free[a], ys, lane, m_warp, n0);
+        epilogue_tile<false, kYBufs>(p, &map_y, tmem + a * 256 + lane_off, &sh->sfreg_free[a], ys, ybuf, sh->bias,
+                                     lane, m_warp, n0);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh->acc_empty[a]);
@@ -590,13 +624,29 @@ int num_sms() {
   return n;
 }
 
+using K2Kernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                         const CUtensorMap, const K2Params);
+
+// The two instantiations: long K (4 stages, one Y buffer per epilogue warp)
+// and short K (3 stages, a ring of 4 Y buffers per warp).
+struct K2Config {
+  K2Kernel fn;
+  size_t smem;
+  int id;
+};
+K2Config k2_config(bool short_k) {
+  if (short_k) return {gemm_w4a4_kernel<3, 4>, 1024 + 3 * static_cast<size_t>(kStage) + sizeof(K2Shared<3, 4>), 1};
+  return {gemm_w4a4_kernel<4, 1>, 1024 + 4 * static_cast<size_t>(kStage) + sizeof(K2Shared<4, 1>), 0};
+}
+
 // Clusters of S CTAs of this kernel that fit on the device at once (cached
-// per device and S).
-int max_active_clusters(int S, size_t smem) {
-  static int cache[64][kMaxSplit + 1] = {};
+// per device, configuration and S).
+int max_active_clusters(const K2Config& kc, int S) {
+  static int cache[64][2][kMaxSplit + 1] = {};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && cache[dev][S]) return cache[dev][S];
+  if (dev >= 0 && dev < 64 && cache[dev][kc.id][S]) return cache[dev][kc.id][S];
+  const size_t smem = kc.smem;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(S, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -609,11 +659,11 @@ int max_active_clusters(int S, size_t smem) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, gemm_w4a4_kernel, &cfg) != cudaSuccess || n < 1) {
+  if (cudaOccupancyMaxActiveClusters(&n, kc.fn, &cfg) != cudaSuccess || n < 1) {
     cudaGetLastError();
     n = -1;  // cached as "does not fit"
   }
-  if (dev >= 0 && dev < 64) cache[dev][S] = n;
+  if (dev >= 0 && dev < 64) cache[dev][kc.id][S] = n;
   return n;
 }
 
@@ -622,12 +672,12 @@ int max_active_clusters(int S, size_t smem) {
 // tile is its longest split (the last split also runs the slab, one stage's
 // worth of MMAs each) plus about two K tiles for the reduction; every tile's
 // cluster must be resident at once.  Ties go to the smaller split.
-int choose_ksplit(int tiles, int kt, int slab, size_t smem) {
+int choose_ksplit(const K2Config& kc, int tiles, int kt, int slab) {
   if (2 * tiles > num_sms()) return 1;
   int best = 1;
   long best_cost = kt + slab;
   for (int S = 2; S <= std::min(kMaxSplit, kt); ++S) {
-    if (max_active_clusters(S, smem) < tiles) continue;
+    if (max_active_clusters(kc, S) < tiles) continue;
     const int base = kt / S, rem = kt % S;
     const long cost = std::max(base + (rem ? 1 : 0), base + slab) + 2;
     if (cost < best_cost) {
@@ -660,8 +710,12 @@ svdq_status launch_gemm_w4a4(const GemmArgs& a, cudaStream_t stream) {
   p.Y = static_cast<uint16_t*>(a.Y);
   // N % 16 == 0, so every 16-column piece starts 32 bytes after the last
   p.y32 = (reinterpret_cast<uintptr_t>(a.Y) & 31u) == 0;
-  // a tile of at least 8 K steps (K >= 1792) hides the staged epilogue of the one before
-  p.tma_y = p.kt + p.slab >= 8 ? 1 : 0;
+  // A tile of at least 8 K steps (K >= 1792) hides the staged epilogue of the
+  // one before; shorter tiles are epilogue-bound and take the configuration
+  // with fewer stages and a ring of Y buffers, whose TMA stores overlap.
+  const bool short_k = p.kt + p.slab < 8;
+  const K2Config kc = k2_config(short_k);
+  p.tma_y = 1;
   p.err = a.err ? a.err : device_error_word();
   p.wait_ns = wait_limit_ns();
   if (!p.err) return fail(SVDQ_ERR_CUDA, "device error word unavailable");
@@ -683,20 +737,23 @@ svdq_status launch_gemm_w4a4(const GemmArgs& a, cudaStream_t stream) {
                     CU_TENSOR_MAP_SWIZZLE_64B);
   if (st != SVDQ_OK) return st;
 
-  const size_t smem = 1024 + static_cast<size_t>(kStages) * kStage + sizeof(K2Shared);
-  static bool attr_set[64] = {};  // per device: the attribute is set on the current one
+  const size_t smem = kc.smem;
+  static bool attr_set[64] = {};  // per device: the attributes are set on the current one
   int cur_dev = 0;
   SVDQ_CUDA_TRY(cudaGetDevice(&cur_dev));
   if (cur_dev < 0 || cur_dev >= 64 || !attr_set[cur_dev]) {
-    SVDQ_CUDA_TRY(cudaFuncSetAttribute(gemm_w4a4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));
+    for (int v = 0; v < 2; ++v) {
+      const K2Config c = k2_config(v == 1);
+      SVDQ_CUDA_TRY(cudaFuncSetAttribute(c.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(c.smem)));
+    }
     if (cur_dev >= 0 && cur_dev < 64) attr_set[cur_dev] = true;
   }
   const int tiles = p.mtiles * p.ntiles;
   if (a.ksplit > 0) {
     p.ksplit = std::min(std::min(a.ksplit, kMaxSplit), p.kt);
-    if (p.ksplit > 1 && max_active_clusters(p.ksplit, smem) < tiles) p.ksplit = 1;
+    if (p.ksplit > 1 && max_active_clusters(kc, p.ksplit) < tiles) p.ksplit = 1;
   } else {
-    p.ksplit = choose_ksplit(tiles, p.kt, p.slab, smem);
+    p.ksplit = choose_ksplit(kc, tiles, p.kt, p.slab);
   }
 
   cudaLaunchConfig_t cfg = {};
@@ -713,7 +770,7 @@ svdq_status launch_gemm_w4a4(const GemmArgs& a, cudaStream_t stream) {
   attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = p.ksplit > 1 ? 2 : 1;
-  SVDQ_CUDA_TRY(cudaLaunchKernelEx(&cfg, gemm_w4a4_kernel, map_xq, *a.map_wq_256, map_t, map_l2, map_y, p));
+  SVDQ_CUDA_TRY(cudaLaunchKernelEx(&cfg, kc.fn, map_xq, *a.map_wq_256, map_t, map_l2, map_y, p));
   return SVDQ_OK;
 }
 
