@@ -271,8 +271,12 @@ svdq_status svdq_forward_norm(const svdq_weights* w, const void* Z_bf16, int M, 
                               size_t workspace_bytes, void* stream);
 
 /*
- * Both kernels back to back.  `workspace` is device memory of at least
- * svdq_forward_workspace_bytes(w, M) bytes holding xq, xsf and T.
+ * The layer on device buffers.  For a few tokens (NVFP4 handle, 1 <= M <= 16,
+ * rank + LoRA ranks <= 64) it runs as one kernel whose CTAs quantize the
+ * activations they need and compute the low-rank branch themselves (see
+ * svdq_debug_forward_small_m); otherwise it is both kernels back to back.
+ * `workspace` is device memory of at least svdq_forward_workspace_bytes(w, M)
+ * bytes holding xq, xsf and T (unused by the one-kernel layer).
  */
 svdq_status svdq_forward(const svdq_weights* w, const void* X_bf16, int M, void* Y_bf16,
                          void* workspace, size_t workspace_bytes, void* stream);
@@ -393,6 +397,21 @@ svdq_status svdq_debug_launch_stalled_act(const svdq_weights* w, const void* X_b
  */
 svdq_status svdq_debug_linear_w4a4_ksplit(const svdq_weights* w, const void* xq, const void* xsf,
                                           const void* T, int M, void* Y_bf16, int ksplit, void* stream);
+
+/*
+ * Test hook: the one-kernel layer that svdq_forward runs for a few tokens
+ * (NVFP4 handle, 1 <= M <= 16, rank + LoRA ranks <= 64), with its split of K
+ * over a cluster fixed to `ksplit` CTAs per 128 output features (0 = the
+ * automatic choice; a split whose clusters would not all be resident at once
+ * is lowered).  Each CTA quantizes the activations of its K range itself (the
+ * same NVFP4 codec as svdq_quantize_act_lowrank_down), computes its share of
+ * T = X L1' and applies L2 to it, and the splits' fp32 partials of Y are
+ * summed in split order.  SVDQ_ERR_INVALID_ARG for other shapes or ksplit
+ * outside [0, 8].
+ *   X_bf16  device, M x K bf16          Y_bf16  device, M x N bf16
+ */
+svdq_status svdq_debug_forward_small_m(const svdq_weights* w, const void* X_bf16, int M, void* Y_bf16,
+                                       int ksplit, void* stream);
 
 /*
  * Device self-test of the NVFP4 group encoder's exact shortcuts (both kernels

@@ -75,6 +75,7 @@ _SIGS = {
                                ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i)]),
     "svdq_debug_launch_stalled_act": (_i, [_vp, _vp, _i, _vp, _vp, _vp, _vp]),
     "svdq_debug_linear_w4a4_ksplit": (_i, [_vp, _vp, _vp, _vp, _i, _vp, _i, _vp]),
+    "svdq_debug_forward_small_m": (_i, [_vp, _vp, _i, _vp, _i, _vp]),
     "svdq_last_error": (ctypes.c_char_p, []),
     "svdq_version": (ctypes.c_char_p, []),
 }
@@ -225,6 +226,11 @@ def svdq_debug_linear_w4a4_ksplit(w: Weights, xq, xsf, T, M: int, Y: torch.Tenso
     _check(_lib.svdq_debug_linear_w4a4_ksplit(w.handle, _dev(xq, "xq"), _dev(xsf, "xsf"), _dev(T, "T"), M,
                                               _dev(Y, "Y"), ksplit, _stream(stream)),
            "svdq_debug_linear_w4a4_ksplit")
+
+
+def svdq_debug_forward_small_m(w: Weights, X: torch.Tensor, Y: torch.Tensor, ksplit: int = 0, stream=None) -> None:
+    _check(_lib.svdq_debug_forward_small_m(w.handle, _dev(X, "X"), X.shape[0], _dev(Y, "Y"), ksplit, _stream(stream)),
+           "svdq_debug_forward_small_m")
 
 
 def svdq_forward(w: Weights, X: torch.Tensor, Y: torch.Tensor, workspace: torch.Tensor, stream=None) -> None:

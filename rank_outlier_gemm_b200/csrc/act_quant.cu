@@ -157,20 +157,37 @@ __global__ void __launch_bounds__(kThreads, 2) act_quant_lowrank_kernel(
       tma_prefetch_desc(&map_x);
       if (lowrank) tma_prefetch_desc(&map_l1);
       const uint32_t bytes = kXTile + (lowrank ? p.l1_tile : 0u) + kAux;
-      int issued = 0;
-      for (int i = 0; i < nt; ++i) {
-        const int s = i % kStages;
-        const uint32_t ph = (i / kStages) & 1;
-        if (!wait_bounded(&sh->empty[s], ph ^ 1, wc)) break;
+      // A stage's loads come in two halves: the layer's own constants (L1'
+      // tile, smoothing multipliers), which no kernel of the forward pass
+      // writes, and X (with the norm front end's a and c), which the kernel
+      // ahead may produce.  The first stages' constants go out before the
+      // wait for that kernel (a programmatic launch lets this kernel start
+      // while the one ahead finishes).
+      auto consts = [&](int i, int s) {
         mbar_arrive_expect_tx(&sh->full[s], bytes);
         const int k0 = (t0 + i) * 64;
-        tma_load_2d(xs + s * kXTile, &map_x, &sh->full[s], k0, m0);
         if (lowrank) tma_load_2d(l1s + s * p.l1_tile, &map_l1, &sh->full[s], k0, 0);
         bulk_load(invs + s * kAux, p.inv_lam + k0, kInvTile, &sh->full[s]);
+      };
+      auto acts = [&](int i, int s) {
+        const int k0 = (t0 + i) * 64;
+        tma_load_2d(xs + s * kXTile, &map_x, &sh->full[s], k0, m0);
         if (kNorm) {
           bulk_load(invs + s * kAux + kInvTile, p.norm_a + k0, kInvTile, &sh->full[s]);
           bulk_load(invs + s * kAux + 2 * kInvTile, p.norm_c + k0, kInvTile, &sh->full[s]);
         }
+      };
+      const int npre = min(kStages, nt);
+      for (int i = 0; i < npre; ++i) consts(i, i);
+      grid_dep_wait();  // X comes from the kernel ahead, which may still read xq, xsf and T
+      for (int i = 0; i < npre; ++i) acts(i, i);
+      int issued = npre;
+      for (int i = npre; i < nt; ++i) {
+        const int s = i % kStages;
+        const uint32_t ph = (i / kStages) & 1;
+        if (!wait_bounded(&sh->empty[s], ph ^ 1, wc)) break;
+        consts(i, s);
+        acts(i, s);
         issued = i + 1;
       }
       if (sh->abort) {  // let copies in flight land before the buffers are reused
@@ -199,6 +216,7 @@ __global__ void __launch_bounds__(kThreads, 2) act_quant_lowrank_kernel(
     const int h = lane & 1;                              // columns [32h, 32h + 32) of the tile
     const int m = m0 + row;
     float mu = 0.0f, rstd = 0.0f;
+    if (kNorm) grid_dep_wait();  // the statistics come from the kernel ahead
     if (kNorm && m < p.M) {
       const float2 st = p.stats[m];
       mu = st.x;
@@ -501,13 +519,17 @@ svdq_status launch_act_quant(const ActArgs& a, cudaStream_t stream) {
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  // a programmatic dependent of the kernel ahead: set-up and constant loads
+  // overlap its tail; everything it may produce or still read waits for it
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 1;
   attr[0].val.clusterDim.y = splits;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   SVDQ_CUDA_TRY(cudaLaunchKernelEx(&cfg, k1_kernel(a.int4 != 0, norm), map_x, map_l1, p));
   return SVDQ_OK;
 }

@@ -528,6 +528,17 @@ svdq_status svdq_linear_w4a4(const svdq_weights* w, const void* xq, const void* 
   return launch_gemm_w4a4(a, static_cast<cudaStream_t>(stream));
 }
 
+svdq_status svdq_debug_forward_small_m(const svdq_weights* w, const void* X_bf16, int M, void* Y_bf16, int ksplit,
+                                       void* stream) {
+  if (ksplit < 0 || ksplit > 8) return fail(SVDQ_ERR_INVALID_ARG, "ksplit=%d must be in [0, 8]", ksplit);
+  SVDQ_TRY(check_runtime(w, M));
+  SVDQ_TRY(check_dev_ptr(X_bf16, "X"));
+  SVDQ_TRY(check_dev_ptr(Y_bf16, "Y"));
+  if (!small_m_supported(M, w->r_pad, w->format))
+    return fail(SVDQ_ERR_INVALID_ARG, "the fused small-M layer takes NVFP4 handles, M <= 16 and rank <= 64");
+  return launch_small_m_for(w, X_bf16, M, Y_bf16, ksplit, nullptr, static_cast<cudaStream_t>(stream));
+}
+
 svdq_status svdq_debug_linear_w4a4_ksplit(const svdq_weights* w, const void* xq, const void* xsf, const void* T,
                                           int M, void* Y_bf16, int ksplit, void* stream) {
   if (ksplit < 1 || ksplit > 8) return fail(SVDQ_ERR_INVALID_ARG, "ksplit=%d must be in [1, 8]", ksplit);
@@ -573,6 +584,11 @@ svdq_status svdq_forward(const svdq_weights* w, const void* X_bf16, int M, void*
   if (workspace_bytes < svdq_forward_workspace_bytes(w, M))
     return fail(SVDQ_ERR_INVALID_ARG, "workspace has %zu bytes, needs %zu", workspace_bytes,
                 svdq_forward_workspace_bytes(w, M));
+  if (small_m_preferred(M, w->N, w->K, w->r_pad, w->format)) {
+    SVDQ_TRY(check_dev_ptr(X_bf16, "X"));
+    SVDQ_TRY(check_dev_ptr(Y_bf16, "Y"));
+    return launch_small_m_for(w, X_bf16, M, Y_bf16, 0, nullptr, static_cast<cudaStream_t>(stream));
+  }
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   uint8_t* xq = ws;
   uint8_t* xsf = xq + up256(svdq_act_codes_bytes(M, w->K));

@@ -160,6 +160,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_int4_kernel(
 
   const uint32_t warp = warp_id(), lane = lane_id();
   const int ntiles_total = p.mtiles * p.ntiles;
+  // the next layer's activation kernel may launch now (it waits for this grid
+  // before touching X or the activation buffers)
+  grid_dep_launch_dependents();
   const int per_tile = p.slab + p.groups;
 
   if (threadIdx.x == 0) {

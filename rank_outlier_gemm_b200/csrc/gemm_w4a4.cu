@@ -291,6 +291,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
   const int nslab = split == S - 1 ? p.slab : 0;
   const int per_tile = nslab + kt_base + (split < kt_rem ? 1 : 0);
   float* part = reinterpret_cast<float*>(smem);  // split-K partials, after the tile's MMAs
+  // the next layer's activation kernel may launch now and take SMs as this
+  // grid's CTAs retire; it waits for this grid before touching X, xq, xsf or T
+  grid_dep_launch_dependents();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {

@@ -92,6 +92,9 @@ extern "C" svdq_status svdq_forward_noalloc(const svdq_weights* w, const void* X
   DeviceScratch d;
   st = scratch_for_current_device(&d);
   if (st != SVDQ_OK) return st;
+  // a few tokens: the one-kernel layer, which keeps no intermediates in memory
+  if (small_m_preferred(M, w->N, w->K, w->r_pad, w->format))
+    return launch_small_m_for(w, X_bf16, M, Y_bf16, 0, d.err, static_cast<cudaStream_t>(stream));
 
   uint8_t* xq = d.base;
   uint8_t* xsf = xq + codes;

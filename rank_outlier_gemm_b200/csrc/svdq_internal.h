@@ -86,6 +86,29 @@ struct GemmArgs {
 };
 svdq_status launch_gemm_w4a4(const GemmArgs& a, cudaStream_t stream);
 
+// The fused single-kernel layer for M <= 16 tokens (NVFP4, rank <= 64).
+struct SmallMArgs {
+  int M, N, K, r_pad;
+  const void* X;                   // device bf16 [M, K]
+  const CUtensorMap* map_wq_128;   // weight codes, box rows 128
+  const CUtensorMap* map_l1;       // L1'^T [r_pad, K] bf16, box 64 x r_pad
+  const CUtensorMap* map_l2_128;   // L2^T/alpha_w [N, r_pad] bf16, box 32 x 128
+  const uint8_t* wsf;              // weight scales (atom layout)
+  const float* inv_lam;            // device [K]
+  const float* bias;               // device [round_up(N, 256)]
+  float alpha_w;
+  void* Y;                         // device bf16 [M, N]
+  int ksplit = 0;                  // CTAs per 128-row tile along K (0 = automatic)
+  int* err = nullptr;
+};
+bool small_m_supported(int M, int r_pad, int format);
+// small_m_supported and expected to beat the two-kernel path on this shape
+bool small_m_preferred(int M, int N, int K, int r_pad, int format);
+svdq_status launch_small_m(const SmallMArgs& a, cudaStream_t stream);
+// launch_small_m for a weights handle (ksplit 0 = automatic; err nullptr = the device's word)
+svdq_status launch_small_m_for(const svdq_weights* w, const void* X, int M, void* Y, int ksplit, int* err,
+                               cudaStream_t stream);
+
 struct GemmInt4Args {
   int M, N, K, r_pad;
   const void* xq;           // device [M, K/2] packed INT4

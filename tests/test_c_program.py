@@ -56,6 +56,7 @@ int main(void) {
       svdq_weights_export(nw, NULL, NULL, NULL, NULL, NULL, NULL, NULL),
       svdq_debug_launch_stalled_act(nw, NULL, 1, NULL, NULL, NULL, NULL),
       svdq_debug_linear_w4a4_ksplit(nw, NULL, NULL, NULL, 1, NULL, 2, NULL),
+      svdq_debug_forward_small_m(nw, NULL, 1, NULL, 0, NULL),
       svdq_act_row_stats(NULL, 1, 64, 1e-6f, NULL, NULL),
       svdq_search_alpha(NULL, NULL, 1, NULL, 16, 64, NULL, 0, &o, NULL, errs, &n),
       svdq_selftest_codec(NULL),
