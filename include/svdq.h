@@ -271,12 +271,8 @@ svdq_status svdq_forward_norm(const svdq_weights* w, const void* Z_bf16, int M, 
                               size_t workspace_bytes, void* stream);
 
 /*
- * The layer on device buffers.  For a few tokens (NVFP4 handle, 1 <= M <= 16,
- * rank + LoRA ranks <= 64) it runs as one kernel whose CTAs quantize the
- * activations they need and compute the low-rank branch themselves (see
- * svdq_debug_forward_small_m); otherwise it is both kernels back to back.
- * `workspace` is device memory of at least svdq_forward_workspace_bytes(w, M)
- * bytes holding xq, xsf and T (unused by the one-kernel layer).
+ * Both kernels back to back.  `workspace` is device memory of at least
+ * svdq_forward_workspace_bytes(w, M) bytes holding xq, xsf and T.
  */
 svdq_status svdq_forward(const svdq_weights* w, const void* X_bf16, int M, void* Y_bf16,
                          void* workspace, size_t workspace_bytes, void* stream);
@@ -399,8 +395,10 @@ svdq_status svdq_debug_linear_w4a4_ksplit(const svdq_weights* w, const void* xq,
                                           const void* T, int M, void* Y_bf16, int ksplit, void* stream);
 
 /*
- * Test hook: the one-kernel layer that svdq_forward runs for a few tokens
- * (NVFP4 handle, 1 <= M <= 16, rank + LoRA ranks <= 64), with its split of K
+ * The layer as one kernel for a few tokens (NVFP4 handle, 1 <= M <= 16,
+ * rank + LoRA ranks <= 64), kept beside the two-kernel path as a measured
+ * alternative (on B200 it is no faster, so svdq_forward does not use it), with
+ * its split of K
  * over a cluster fixed to `ksplit` CTAs per 128 output features (0 = the
  * automatic choice; a split whose clusters would not all be resident at once
  * is lowered).  Each CTA quantizes the activations of its K range itself (the

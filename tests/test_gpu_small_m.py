@@ -1,6 +1,6 @@
 """GPU parity of the one-kernel layer for a few tokens (M <= 16, NVFP4 handle,
-rank + LoRA ranks <= 64; svdq_forward takes it where each CTA has at most 3
-K tiles, svdq_debug_forward_small_m always), through the C ABI.
+rank + LoRA ranks <= 64; reached through svdq_debug_forward_small_m, while
+svdq_forward keeps the faster two-kernel path), through the C ABI.
 
 That kernel quantizes the activations inside the GEMM's CTAs, computes each
 CTA's share of the down-projection T = X L1' on the tensor cores, applies L2
@@ -112,8 +112,9 @@ def test_rank0_and_rank64_handles():
 
 
 def test_fallback_above_the_limits():
-    """M = 17 and rank 64 + LoRA 16 (r_pad 80) take the two-kernel path, which
-    svdq_debug_forward_small_m refuses; svdq_forward still matches the oracle."""
+    """M = 17 and rank 64 + LoRA 16 (r_pad 80) are outside the one-kernel
+    layer, which svdq_debug_forward_small_m refuses; svdq_forward matches the
+    oracle there."""
     L = G.lib()
     case, t, prep = _small_case("M16_N3072", 17)
     w, ref = _lora_handle(case, t, prep)
