@@ -61,10 +61,10 @@ def peaks():
 # kernel source the counters were taken on; counters of another source are stale
 # and not reported.
 K2_TRAFFIC = {
-    "source_sha256": "4aaa299b83115cf162973296dfe5b0fff5da7d2f120f9935a301ac7e05427a3e",
+    "source_sha256": "08720887c846a6aa8f04d016644c3b8d285b00021466ff14c7beb0b58ba4afc3",
     # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum: read + write per launch
-    "bytes_per_launch": {"attn_out": 14127104 + 16384, "qkv": 25167104 + 32058880,
-                         "mlp_up": 30682112 + 59258624, "mlp_down": 55453440 + 5070592},
+    "bytes_per_launch": {"attn_out": 14127360 + 17920, "qkv": 25181952 + 32743168,
+                         "mlp_up": 30683648 + 59607296, "mlp_down": 55538688 + 5762560},
 }
 
 
@@ -769,6 +769,50 @@ def run_reference(args):
     print(json.dumps(out))
 
 
+def run_layer_only(args):
+    """Profiling mode: one configured layer (``cfg/name`` or ``cfg/name:M``),
+    library-prepared weights (LoRA attached where the configuration has one),
+    ``--warmup`` + ``--steps`` launches of the activation kernel and the GEMM
+    (``--kernel act|gemm|both``: the GEMM-only mode runs the activation kernel
+    once first), and one JSON line with the mean device time per launch pair.
+    For ncu captures of a single kernel on a chosen shape."""
+    import torch
+    import rank_outlier_gemm_b200 as L
+
+    lab, _, m = args.layer_only.partition(":")
+    cfg, name = lab.split("/")
+    c = [x for x in config_cases(cfg) if x.name == name][0]
+    M = int(m) if m else c.M
+    t = make_layer_inputs(c, M=M)
+    w = L.svdq_prepare_weights(t.W_bits, t.act_absmax, t.bias_bits, rank=c.rank, fmt=args.format)
+    if c.lora_rank:
+        L.svdq_attach_lora(w, t.lora_A_bits, t.lora_B_bits, t.lora_scale)
+    X = torch.from_numpy(t.X_bits.view(np.int16).copy()).view(torch.bfloat16).cuda()
+    xq, xsf, T = L.act_buffers(w, M)
+    Y = torch.empty((M, c.N), dtype=torch.bfloat16, device="cuda")
+
+    def one():
+        if args.kernel in ("act", "both"):
+            L.svdq_quantize_act_lowrank_down(w, X, xq, xsf, T)
+        if args.kernel in ("gemm", "both"):
+            L.svdq_linear_w4a4(w, xq, xsf, T, M, Y)
+
+    if args.kernel == "gemm":
+        L.svdq_quantize_act_lowrank_down(w, X, xq, xsf, T)
+    for _ in range(args.warmup):
+        one()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(args.steps):
+        one()
+    b.record()
+    torch.cuda.synchronize()
+    assert L.svdq_check_device_errors() == 0
+    print(json.dumps({"layer": f"{lab} M={M} K={c.K} N={c.N}", "kernel": args.kernel,
+                      "us_per_launch": 1e3 * a.elapsed_time(b) / args.steps}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -784,7 +828,16 @@ def main():
     ap.add_argument("--layers", default="", help="comma-separated subset of the FLUX layers (profiling)")
     ap.add_argument("--format", choices=["nvfp4", "int4"], default="nvfp4",
                     help="4-bit format of the timed step (INT4: the variant with group-64 bf16 scales)")
+    ap.add_argument("--layer-only", default="",
+                    help="profiling: time one configured layer, cfg/name[:M] (e.g. small_m_lora/M16_N12288:16)")
+    ap.add_argument("--kernel", choices=["act", "gemm", "both"], default="both",
+                    help="with --layer-only: which kernel(s) to launch")
     args = ap.parse_args()
+    if args.layer_only:
+        if args.warmup < 3:
+            ap.error("--warmup must be >= 3")
+        run_layer_only(args)
+        return
     global LAYER_FILTER
     LAYER_FILTER = [x for x in args.layers.split(",") if x] or None
     if args.warmup < 3:
