@@ -56,15 +56,16 @@ def peaks():
                 "hbm": FALLBACK_HBM, "source": "fallback"}
 
 
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of
-# gemm_w4a4_kernel on this workload, from one ncu capture, with the SHA-256 of the
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the
+# step's GEMM (gemm_w4a4_kernel for K = 3072, the CTA-pair gemm_w4a4_pair_kernel
+# for K = 12288) on this workload, from one ncu capture, with the SHA-256 of the
 # kernel source the counters were taken on; counters of another source are stale
 # and not reported.
 K2_TRAFFIC = {
-    "source_sha256": "08720887c846a6aa8f04d016644c3b8d285b00021466ff14c7beb0b58ba4afc3",
+    "source_sha256": "9482a6cdf741aef42773aed4d9c3fa2f865809d300b8ffab3cc1fa8a2e20917c",
     # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum: read + write per launch
-    "bytes_per_launch": {"attn_out": 14127360 + 17920, "qkv": 25181952 + 32743168,
-                         "mlp_up": 30683648 + 59607296, "mlp_down": 55538688 + 5762560},
+    "bytes_per_launch": {"attn_out": 14127616 + 17152, "qkv": 25167872 + 32066816,
+                         "mlp_up": 30682624 + 59291392, "mlp_down": 55654144 + 6521344},
 }
 
 
@@ -665,7 +666,8 @@ def run_ours(args):
             "lowrank_overhead_vs_rank0": overhead,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
                          "frac": achieved / fp4_peak, "traffic": traffic, "traffic_note": traffic_note,
-                         "kernel": "gemm_int4_kernel" if args.format == "int4" else "gemm_w4a4_kernel",
+                         "kernel": "gemm_int4_kernel" if args.format == "int4" else
+                         "gemm_w4a4_kernel (K = 3072 layers), gemm_w4a4_pair_kernel (K = 12288)",
                          "peak_source": peak_src,
                          "frac_of_datasheet_9pf": achieved / 9000.0},
             "gpu_launches": 2 * nl * args.steps,

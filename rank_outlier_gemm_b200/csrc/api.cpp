@@ -99,6 +99,23 @@ svdq_status make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType
   return SVDQ_OK;
 }
 
+svdq_status make_tmap_3d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, const uint64_t dims[3],
+                         const uint64_t strides[2], const uint32_t box[3]) {
+  auto fn = encode_fn();
+  if (!fn) return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t d[3] = {dims[0], dims[1], dims[2]};
+  cuuint64_t st[2] = {strides[0], strides[1]};
+  cuuint32_t bx[3] = {box[0], box[1], box[2]};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, dtype, 3, const_cast<void*>(base), d, st, bx, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for a 3-D map [%llu x %llu x %llu]",
+                static_cast<int>(r), static_cast<unsigned long long>(dims[2]),
+                static_cast<unsigned long long>(dims[1]), static_cast<unsigned long long>(dims[0]));
+  return SVDQ_OK;
+}
+
 namespace {
 
 void free_device(svdq_weights* w) {
@@ -237,6 +254,12 @@ svdq_status build_handle(int N, int K, int rank, const float* inv_lam, const uin
   if (st == SVDQ_OK)
     st = make_tmap_2d(&w->map_wq_128, w->d_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, N, K / 2, 128, 128,
                       CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st == SVDQ_OK) {  // scale atoms [npad/128][K/64][512 bytes] as 32-bit words
+    const uint64_t dims[3] = {128, static_cast<uint64_t>(K / 64), static_cast<uint64_t>(npad / 128)};
+    const uint64_t strides[2] = {512, static_cast<uint64_t>(K / 64) * 512};
+    const uint32_t box[3] = {128, 4, 2};
+    st = make_tmap_3d(&w->map_wsf, w->d_wsf, CU_TENSOR_MAP_DATA_TYPE_UINT32, dims, strides, box);
+  }
   if (st != SVDQ_OK) return bail(st);
   *out = w;
   return SVDQ_OK;
@@ -525,6 +548,7 @@ svdq_status svdq_linear_w4a4(const svdq_weights* w, const void* xq, const void* 
   if (w->format == SVDQ_FORMAT_INT4) return launch_int4(w, xq, xsf, T, M, Y_bf16, stream);
   GemmArgs a{M, w->N, w->K, w->r_pad, xq, xsf, T, &w->map_wq_256, &w->map_wq_128, &w->map_l2_256,
              &w->map_l2_128, w->d_wsf, w->d_bias, w->alpha_w, Y_bf16, 0};
+  a.map_wsf = &w->map_wsf;
   return launch_gemm_w4a4(a, static_cast<cudaStream_t>(stream));
 }
 
@@ -550,6 +574,7 @@ svdq_status svdq_debug_linear_w4a4_ksplit(const svdq_weights* w, const void* xq,
   if (w->format == SVDQ_FORMAT_INT4) return launch_int4(w, xq, xsf, T, M, Y_bf16, stream);  // no split-K
   GemmArgs a{M, w->N, w->K, w->r_pad, xq, xsf, T, &w->map_wq_256, &w->map_wq_128, &w->map_l2_256,
              &w->map_l2_128, w->d_wsf, w->d_bias, w->alpha_w, Y_bf16, ksplit};
+  a.map_wsf = &w->map_wsf;
   return launch_gemm_w4a4(a, static_cast<cudaStream_t>(stream));
 }
 

@@ -198,8 +198,8 @@ __device__ __forceinline__ void store_chunk_direct(const uint32_t (&r)[32], cons
 // chunks 3-7, each chunk's TMEM load in flight while the one before is stored.
 template <bool kTma, int kYBufs>
 __device__ __forceinline__ void epilogue_tile(const K2Params& p, const CUtensorMap* map_y, uint32_t acc,
-                                              uint64_t* sfreg_free, uint8_t (*ys)[2048], int& ybuf,
-                                              const float* bias_s, uint32_t lane, int m_warp, int n0) {
+                                              uint64_t* sfreg_free, uint64_t* sfreg_free2, uint8_t (*ys)[2048],
+                                              int& ybuf, const float* bias_s, uint32_t lane, int m_warp, int n0) {
   auto put = [&](const uint32_t(&rr)[32], int c) {
     if constexpr (kTma)
       store_chunk_tma<kYBufs>(rr, p, map_y, ys, ybuf, bias_s + 32 * c, lane, m_warp, n0 + 32 * c);
@@ -221,6 +221,12 @@ __device__ __forceinline__ void epilogue_tile(const K2Params& p, const CUtensorM
 #pragma unroll
   for (int c = 3; c < kBN / 32; ++c) {
     tmem_ld_wait_regs(nx);
+    if (sfreg_free2 && c == 4) {
+      // columns 96..159 read: a third scale slot (columns 96..143) may go there
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sfreg_free2);
+    }
     uint32_t cur[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) cur[i] = nx[i];
@@ -588,11 +594,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
         continue;
       }
       if (tma)
-        epilogue_tile<true, kYBufs>(p, &map_y, tmem + a * 256 + lane_off, &sh->sfreg_free[a], ys, ybuf, sh->bias,
-                                    lane, m_warp, n0);
+        epilogue_tile<true, kYBufs>(p, &map_y, tmem + a * 256 + lane_off, &sh->sfreg_free[a], nullptr, ys, ybuf,
+                                    sh->bias, lane, m_warp, n0);
       else
-        epilogue_tile<false, kYBufs>(p, &map_y, tmem + a * 256 + lane_off, &sh->sfreg_free[a], ys, ybuf, sh->bias,
-                                     lane, m_warp, n0);
+        epilogue_tile<false, kYBufs>(p, &map_y, tmem + a * 256 + lane_off, &sh->sfreg_free[a], nullptr, ys, ybuf,
+                                     sh->bias, lane, m_warp, n0);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh->acc_empty[a]);
@@ -616,6 +622,349 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_w4a4_kernel(
   }
 }
 
+// ------------------------------------------------------------------ CTA pair
+// Many output tiles: a cluster of two CTAs takes 256 x 256 tiles, each MMA an
+// M = 256 pair operation issued by rank 0.  Each CTA stages its own 128 rows
+// of the activation codes and 128 of the 256 weight rows, so a K tile brings
+// 38 KB into each SM instead of 54 KB and five stages fit where four did; each
+// CTA's TMEM holds its 128 accumulator rows and the scale atoms of its rows and
+// of all 256 weight rows (the layout the pair MMA reads in both CTAs).
+// Every load completes on a barrier of its own CTA, so each CTA can account
+// for its copies in flight; what the leader's MMA issuer needs of the peer
+// (its operands landed, its scale slots filled, its accumulator rows drained)
+// reaches it as arrivals on the leader's barriers, and the leader's commits
+// arrive on the same barrier in both CTAs.  Three scale slots: the MMAs of a
+// K tile wait only for the slot filled after the K tile three back retired.
+constexpr int kPBTile = 128 * 128;                             // this CTA's 128 weight rows x 128 bytes
+constexpr int kPStage = kATile + kPBTile + kSfa + kSfb;        // 38 KB
+constexpr int kPSlots = 3;                                     // 3 x 48 = 144 columns of the idle accumulator
+static_assert(kPStage % 1024 == 0, "stage buffers keep 1024-byte alignment");
+
+template <int kStages, int kYBufs>
+struct K2PairShared {
+  alignas(1024) uint8_t ystage[4][kYBufs][2048];
+  float bias[kBN];
+  uint64_t full[kStages];       // this CTA's bytes of the stage (operands, scales, T, L2)
+  uint64_t empty[kStages];      // the leader's MMA commit
+  uint64_t peer_full[kStages];  // leader: the peer's bytes of the stage have landed
+  uint64_t sf_full[kPSlots];    // leader: the pair's eight scale-writer warps
+  uint64_t sf_empty[kPSlots];   // the leader's MMA commit
+  uint64_t acc_full[2];         // the leader's MMA commit
+  uint64_t acc_empty[2];        // leader: the pair's eight epilogue warps
+  uint64_t sfreg_free[2];       // this CTA's epilogue warps have read columns 0..95
+  uint64_t sfreg_free2[2];      // ... and columns 96..159
+  uint64_t done;                // leader: every MMA has retired
+  uint32_t tmem_base;
+  int abort;
+  int epi_stop;
+};
+
+// p.mtiles counts 256-row pair tiles here.
+constexpr int kPThreads = 352;  // the 320 of the single-CTA kernel plus a weight-side producer warp
+template <int kStages, int kYBufs>
+__global__ void __launch_bounds__(kPThreads, 1) gemm_w4a4_pair_kernel(
+    const __grid_constant__ CUtensorMap map_xq, const __grid_constant__ CUtensorMap map_wq,
+    const __grid_constant__ CUtensorMap map_t, const __grid_constant__ CUtensorMap map_l2,
+    const __grid_constant__ CUtensorMap map_y, const __grid_constant__ CUtensorMap map_wsf, const K2Params p) {
+  using Shared = K2PairShared<kStages, kYBufs>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Shared* sh = reinterpret_cast<Shared*>(smem + kStages * kPStage);
+  static_assert(offsetof(Shared, ystage) == 0, "Y staging buffers keep the 1024-byte alignment the swizzle needs");
+
+  const uint32_t warp = warp_id(), lane = lane_id();
+  const int rank = static_cast<int>(cluster_ctarank());  // 0 = leader
+  const bool leader = rank == 0;
+  const int ntiles_total = p.mtiles * p.ntiles;
+  const int pair0 = static_cast<int>(blockIdx.x) >> 1, npairs = static_cast<int>(gridDim.x) >> 1;
+  const int per_tile = p.slab + p.kt;
+  grid_dep_launch_dependents();
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sh->full[s], 1);
+      mbar_init(&sh->empty[s], 1);
+      mbar_init(&sh->peer_full[s], 1);
+    }
+    for (int b = 0; b < kPSlots; ++b) {
+      mbar_init(&sh->sf_full[b], 8);
+      mbar_init(&sh->sf_empty[b], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sh->acc_full[b], 1);
+      mbar_init(&sh->acc_empty[b], 8);
+      mbar_init(&sh->sfreg_free[b], 4);
+      mbar_init(&sh->sfreg_free2[b], 4);
+    }
+    mbar_init(&sh->done, 1);
+    sh->abort = 0;
+    sh->epi_stop = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&sh->tmem_base, 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers exist before any cross-CTA arrival
+  tc_fence_after();
+  const WaitCtl wc{p.err, p.wait_ns, &sh->abort};
+  const uint32_t tmem = sh->tmem_base;
+
+  if (warp == 0 || warp == 10) {
+    // ------------------------------------------------------------ producers
+    // Warp 10 issues the weight half of every stage (codes and both 128-row
+    // blocks of scale atoms in one 3-D copy, or L2), which no kernel of the
+    // forward pass writes, and arms the stage's barrier for all its bytes; warp
+    // 0 issues the activation half (codes and scales, or T) once the kernel
+    // ahead has finished.  A thread issuing a copy waits for the copy engine to
+    // take it (~130 cycles each): one thread for all of a stage's copies was
+    // the bound on the K-tile rate.
+    if (lane == 0) {
+      const bool wside = warp == 10;
+      if (wside) {
+        tma_prefetch_desc(&map_wq);
+        tma_prefetch_desc(&map_wsf);
+        if (p.slab) tma_prefetch_desc(&map_l2);
+      } else {
+        tma_prefetch_desc(&map_xq);
+        if (p.slab) tma_prefetch_desc(&map_t);
+        grid_dep_wait();
+      }
+      int it = 0;
+      bool ok = true;
+      for (int t = pair0; ok && t < ntiles_total; t += npairs) {
+        const int m0 = (t % p.mtiles) * 256 + 128 * rank;
+        const int n0 = (t / p.mtiles) * kBN;
+        const int sfa_valid = m0 < p.M ? 1 : 0;
+        for (int k = 0; k < per_tile; ++k, ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = (it / kStages) & 1;
+          if (!wait_bounded(&sh->empty[s], ph ^ 1, wc)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + s * kPStage;
+          if (k >= p.slab) {
+            const int kk = k - p.slab;
+            const int nkb = min(4, p.kb_total - 4 * kk);
+            if (wside) {
+              // a tiled copy counts its whole box, the parts outside the array included
+              mbar_arrive_expect_tx(&sh->full[s], kATile + kPBTile + kSfb + 512u * nkb * sfa_valid);
+              tma_load_2d(st + kATile, &map_wq, &sh->full[s], kk * 128, n0 + 128 * rank);
+              tma_load_3d(st + kATile + kPBTile + kSfa, &map_wsf, &sh->full[s], 0, 4 * kk, n0 / 128);
+            } else {
+              tma_load_2d(st, &map_xq, &sh->full[s], kk * 128, m0);
+              if (sfa_valid)
+                bulk_load(st + kATile + kPBTile, p.xsf + (static_cast<size_t>(m0 / 128) * p.kb_total + 4 * kk) * 512,
+                          512u * nkb, &sh->full[s]);
+            }
+          } else {
+            if (wside) {
+              mbar_arrive_expect_tx(&sh->full[s], kATile + 128 * 64);
+              tma_load_2d(st + kATile, &map_l2, &sh->full[s], 32 * k, n0 + 128 * rank);
+            } else {
+              tma_load_2d(st, &map_t, &sh->full[s], 64 * k, m0);
+            }
+          }
+        }
+      }
+      if (sh->abort) {  // this CTA's copies in flight land before it exits
+        for (int i = max(0, it - kStages); i < it; ++i)
+          wait_drain(&sh->full[i % kStages], (i / kStages) & 1, p.wait_ns);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer (leader)
+    if (leader && lane == 0) {
+      const uint32_t id_fp4 = idesc_nvfp4(256, kBN);
+      const uint32_t id_bf16 = idesc_bf16(256, kBN);
+      const uint32_t stage0 = smem_u32(smem);
+      const uint64_t da0 = desc_kmajor_sw128(stage0);
+      const uint64_t db0 = desc_kmajor_sw128(stage0 + kATile);
+      const uint64_t dl0 = desc_kmajor_sw64(stage0 + kATile);
+      int it = 0, j = 0;
+      int b = 0;
+      uint32_t bph = 0;  // scale slot and the parity of its current fill
+      bool ok = true;
+      for (int t = pair0; ok && t < ntiles_total; t += npairs, ++j) {
+        const int a = j & 1;
+        if (!wait_bounded(&sh->acc_empty[a], ((j >> 1) & 1) ^ 1, wc)) break;
+        tc_fence_after();
+        const uint32_t acc = tmem + a * 256;
+        const uint32_t sf_region = tmem + (a ^ 1) * 256;
+        uint32_t accum = 0;
+        for (int k = 0; k < per_tile; ++k, ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = (it / kStages) & 1;
+          const uint64_t soff = static_cast<uint64_t>(s * (kPStage >> 4));
+          if (k >= p.slab) {
+            const int nkb = min(4, p.kb_total - 4 * (k - p.slab));
+            // both CTAs' writers saw their CTA's bytes of the stage land first
+            if (!wait_bounded(&sh->sf_full[b], bph, wc)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t sfa = sf_region + b * kSfCols;
+            const uint32_t sfb = sfa + 16;
+            const uint64_t adesc = da0 + soff, bdesc = db0 + soff;
+            if (nkb == 4) {
+              mma_nvfp4_pair_x4(acc, adesc, bdesc, id_fp4, sfa, sfb, accum);
+            } else {
+              for (int kb = 0; kb < nkb; ++kb)
+                mma_nvfp4_pair(acc, adesc + 2 * kb, bdesc + 2 * kb, id_fp4, sfa + 4 * kb, sfb + 8 * kb,
+                               kb ? 1u : accum);
+            }
+            accum = 1;
+            mma_commit_both(&sh->sf_empty[b]);
+            mma_commit_both(&sh->empty[s]);
+            if (++b == kPSlots) {
+              b = 0;
+              bph ^= 1;
+            }
+          } else {
+            if (!wait_bounded(&sh->full[s], ph, wc) || !wait_bounded(&sh->peer_full[s], ph, wc)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              if (32 * k + 16 * c >= p.r_pad) break;
+              const uint64_t ldesc = dl0 + soff + 2 * c;
+              mma_bf16_pair(acc, da0 + soff + 4 * c, ldesc, id_bf16, accum);  // T_hi
+              mma_bf16_pair(acc, da0 + soff + 4 * c + 2, ldesc, id_bf16, 1);  // T_lo
+              accum = 1;
+            }
+            mma_commit_both(&sh->empty[s]);
+          }
+        }
+        if (ok) mma_commit_both(&sh->acc_full[a]);
+      }
+      mma_commit_pair_local(&sh->done);
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------------ scale writers
+    const int q = warp & 3;
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    const uint32_t sf_full_l = mapa_shared(smem_u32(&sh->sf_full[0]), 0);
+    const uint32_t peer_full_l = mapa_shared(smem_u32(&sh->peer_full[0]), 0);
+    int it = 0, j = 0;
+    int b = 0;
+    uint32_t bph = 0;
+    bool ok = true;
+    for (int t = pair0; ok && t < ntiles_total; t += npairs, ++j) {
+      const int a = j & 1;
+      const uint32_t sf_region = tmem + (a ^ 1) * 256 + lane_off;
+      bool third_free = false;  // the previous tile's epilogue has read columns 96..159
+      for (int k = 0; k < per_tile; ++k, ++it) {
+        const int s = it % kStages;
+        const uint32_t ph = (it / kStages) & 1;
+        if (!wait_warp(&sh->full[s], ph, wc)) {
+          ok = false;
+          break;
+        }
+        // the peer tells the leader's MMA issuer that its bytes of the stage are in
+        if (!leader && warp == 2 && lane == 0) mbar_arrive_cluster(peer_full_l + 8u * s);
+        if (k < p.slab) continue;
+        const uint8_t* sfa_s = smem + s * kPStage + kATile + kPBTile;
+        const uint8_t* sfb_s = sfa_s + kSfa;
+        uint32_t ra[16], rb[32];
+#pragma unroll
+        for (int kb = 0; kb < 4; ++kb) {
+          const uint4 v = *reinterpret_cast<const uint4*>(sfa_s + kb * 512 + lane * 16);
+          ra[4 * kb] = v.x;
+          ra[4 * kb + 1] = v.y;
+          ra[4 * kb + 2] = v.z;
+          ra[4 * kb + 3] = v.w;
+#pragma unroll
+          for (int nb = 0; nb < 2; ++nb) {
+            const uint4 u = *reinterpret_cast<const uint4*>(sfb_s + nb * 2048 + kb * 512 + lane * 16);
+            rb[8 * kb + 4 * nb] = u.x;
+            rb[8 * kb + 4 * nb + 1] = u.y;
+            rb[8 * kb + 4 * nb + 2] = u.z;
+            rb[8 * kb + 4 * nb + 3] = u.w;
+          }
+        }
+        // the scale slots live in acc[a^1]: before the tile's first store into
+        // a slot, wait until the previous tile's epilogue of this CTA has read it
+        if (k == p.slab && !wait_warp(&sh->sfreg_free[a ^ 1], ((j - 1) >> 1) & 1, wc)) {
+          ok = false;
+          break;
+        }
+        if (b == 2 && !third_free) {
+          if (!wait_warp(&sh->sfreg_free2[a ^ 1], ((j - 1) >> 1) & 1, wc)) {
+            ok = false;
+            break;
+          }
+          third_free = true;
+        }
+        if (!wait_warp(&sh->sf_empty[b], bph ^ 1, wc)) {
+          ok = false;
+          break;
+        }
+        const uint32_t dst = sf_region + b * kSfCols;
+        tmem_st_x16(dst, ra);
+        tmem_st_x32(dst + 16, rb);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(sf_full_l + 8u * b);
+        if (++b == kPSlots) {
+          b = 0;
+          bph ^= 1;
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    const uint32_t acc_empty_l = mapa_shared(smem_u32(&sh->acc_empty[0]), 0);
+    uint8_t(*ys)[2048] = sh->ystage[warp - 6];
+    const int et = static_cast<int>(threadIdx.x) - 6 * 32;
+    int ybuf = 0;
+    int j = 0;
+    for (int t = pair0; t < ntiles_total; t += npairs, ++j) {
+      const int a = j & 1;
+      const int m_warp = (t % p.mtiles) * 256 + 128 * rank + q * 32;
+      const int n0 = (t / p.mtiles) * kBN;
+      const bool tma = p.tma_y && (kYBufs > 1 || t + npairs < ntiles_total);
+      const float2 bpre = __ldg(reinterpret_cast<const float2*>(p.bias + n0) + et);
+      if (!wait_warp(&sh->acc_full[a], (j >> 1) & 1, wc) && lane == 0) sh->epi_stop = 1;
+      epi_bar();
+      const bool stop = sh->epi_stop != 0;
+      if (!stop) reinterpret_cast<float2*>(sh->bias)[et] = bpre;
+      epi_bar();
+      if (stop) break;
+      tc_fence_after();
+      if (tma)
+        epilogue_tile<true, kYBufs>(p, &map_y, tmem + a * 256 + lane_off, &sh->sfreg_free[a], &sh->sfreg_free2[a], ys, ybuf,
+                                    sh->bias, lane, m_warp, n0);
+      else
+        epilogue_tile<false, kYBufs>(p, &map_y, tmem + a * 256 + lane_off, &sh->sfreg_free[a], &sh->sfreg_free2[a], ys, ybuf,
+                                     sh->bias, lane, m_warp, n0);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc_empty_l + 8u * a);
+    }
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1 && leader && lane == 0) wait_drain(&sh->done, 0, p.wait_ns);  // every MMA has retired
+  __syncthreads();
+  cluster_sync_all();  // no cross-CTA arrival or MMA access is still in flight
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, 512);
+  }
+}
+
 int num_sms() {
   static int n = 0;
   if (!n) {
@@ -629,30 +978,44 @@ int num_sms() {
 
 using K2Kernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap,
                          const CUtensorMap, const K2Params);
+using K2PairKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                             const CUtensorMap, const CUtensorMap, const K2Params);
 
 // The two instantiations: long K (4 stages, one Y buffer per epilogue warp)
 // and short K (3 stages, a ring of 4 Y buffers per warp).
 struct K2Config {
-  K2Kernel fn;
+  K2Kernel fn;        // single-CTA kernel (nullptr for the pair kernel)
+  K2PairKernel pfn;   // CTA-pair kernel
   size_t smem;
   int id;
+  const void* entry() const { return fn ? reinterpret_cast<const void*>(fn) : reinterpret_cast<const void*>(pfn); }
 };
 K2Config k2_config(bool short_k) {
-  if (short_k) return {gemm_w4a4_kernel<3, 4>, 1024 + 3 * static_cast<size_t>(kStage) + sizeof(K2Shared<3, 4>), 1};
-  return {gemm_w4a4_kernel<4, 1>, 1024 + 4 * static_cast<size_t>(kStage) + sizeof(K2Shared<4, 1>), 0};
+  if (short_k)
+    return {gemm_w4a4_kernel<3, 4>, nullptr, 1024 + 3 * static_cast<size_t>(kStage) + sizeof(K2Shared<3, 4>), 1};
+  return {gemm_w4a4_kernel<4, 1>, nullptr, 1024 + 4 * static_cast<size_t>(kStage) + sizeof(K2Shared<4, 1>), 0};
 }
+// The CTA-pair kernel: five stages and a ring of four Y buffers per epilogue warp.
+constexpr int kPairStages = 5, kPairYBufs = 4;
+constexpr int kPairMinKTiles = 16;  // K > 3840
+K2Config k2_pair_config() {
+  return {nullptr, gemm_w4a4_pair_kernel<kPairStages, kPairYBufs>,
+          1024 + kPairStages * static_cast<size_t>(kPStage) + sizeof(K2PairShared<kPairStages, kPairYBufs>), 2};
+}
+static_assert(1024 + kPairStages * kPStage + sizeof(K2PairShared<kPairStages, kPairYBufs>) <= 232448,
+              "the pair kernel's shared memory fits one CTA per SM");
 
 // Clusters of S CTAs of this kernel that fit on the device at once (cached
 // per device, configuration and S).
 int max_active_clusters(const K2Config& kc, int S) {
-  static int cache[64][2][kMaxSplit + 1] = {};
+  static int cache[64][3][kMaxSplit + 1] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && cache[dev][kc.id][S]) return cache[dev][kc.id][S];
   const size_t smem = kc.smem;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(S, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(kc.id == 2 ? kPThreads : kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -662,7 +1025,7 @@ int max_active_clusters(const K2Config& kc, int S) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, kc.fn, &cfg) != cudaSuccess || n < 1) {
+  if (cudaOccupancyMaxActiveClusters(&n, kc.entry(), &cfg) != cudaSuccess || n < 1) {
     cudaGetLastError();
     n = -1;  // cached as "does not fit"
   }
@@ -745,9 +1108,10 @@ svdq_status launch_gemm_w4a4(const GemmArgs& a, cudaStream_t stream) {
   int cur_dev = 0;
   SVDQ_CUDA_TRY(cudaGetDevice(&cur_dev));
   if (cur_dev < 0 || cur_dev >= 64 || !attr_set[cur_dev]) {
-    for (int v = 0; v < 2; ++v) {
-      const K2Config c = k2_config(v == 1);
-      SVDQ_CUDA_TRY(cudaFuncSetAttribute(c.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(c.smem)));
+    for (int v = 0; v < 3; ++v) {
+      const K2Config c = v == 2 ? k2_pair_config() : k2_config(v == 1);
+      SVDQ_CUDA_TRY(
+          cudaFuncSetAttribute(c.entry(), cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(c.smem)));
     }
     if (cur_dev >= 0 && cur_dev < 64) attr_set[cur_dev] = true;
   }
@@ -757,6 +1121,41 @@ svdq_status launch_gemm_w4a4(const GemmArgs& a, cudaStream_t stream) {
     if (p.ksplit > 1 && max_active_clusters(kc, p.ksplit) < tiles) p.ksplit = 1;
   } else {
     p.ksplit = choose_ksplit(kc, tiles, p.kt, p.slab);
+  }
+
+  // Many tiles, long K and no split requested: the CTA-pair kernel over
+  // 256 x 256 tiles, one pair per resident cluster of two.  Measured against
+  // the single-CTA kernel (GEMM alone, CUDA-graph replay, us): ahead from 16 K
+  // tiles (FLUX 12288 -> 3072 75.4 vs 79.2, SDXL 10240 -> 1280 23.5 vs 25.2,
+  // PixArt 4608 -> 1152 21.7 vs 22.0), level within noise at 5-12 K tiles
+  // (and behind in the full step, where its clusters of two start later behind
+  // the activation kernel), behind below 4 (SDXL 640-wide: 33.5 vs 31.6).
+  if (a.ksplit == 0 && p.ksplit == 1 && p.kt >= kPairMinKTiles && a.map_wq_128 && a.map_wsf &&
+      (a.r_pad == 0 || a.map_l2_128)) {
+    const K2Config pc = k2_pair_config();
+    const int pairs_fit = max_active_clusters(pc, 2);
+    if (pairs_fit >= 1) {
+      K2Params pp = p;
+      pp.mtiles = (a.M + 255) / 256;
+      const int ptiles = pp.mtiles * pp.ntiles;
+      const CUtensorMap& map_l2_p = a.r_pad > 0 ? *a.map_l2_128 : map_xq;
+      cudaLaunchConfig_t pcfg = {};
+      pcfg.gridDim = dim3(2 * std::min(ptiles, pairs_fit), 1, 1);
+      pcfg.blockDim = dim3(kPThreads, 1, 1);
+      pcfg.dynamicSmemBytes = pc.smem;
+      pcfg.stream = stream;
+      cudaLaunchAttribute pattr[2];
+      pattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      pattr[0].val.programmaticStreamSerializationAllowed = 1;
+      pattr[1].id = cudaLaunchAttributeClusterDimension;
+      pattr[1].val.clusterDim.x = 2;
+      pattr[1].val.clusterDim.y = 1;
+      pattr[1].val.clusterDim.z = 1;
+      pcfg.attrs = pattr;
+      pcfg.numAttrs = 2;
+      SVDQ_CUDA_TRY(cudaLaunchKernelEx(&pcfg, pc.pfn, map_xq, *a.map_wq_128, map_t, map_l2_p, map_y, *a.map_wsf, pp));
+      return SVDQ_OK;
+    }
   }
 
   cudaLaunchConfig_t cfg = {};

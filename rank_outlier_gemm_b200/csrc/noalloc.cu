@@ -113,6 +113,7 @@ extern "C" svdq_status svdq_forward_noalloc(const svdq_weights* w, const void* X
   }
   GemmArgs g{M, w->N, w->K, w->r_pad, xq, xsf, T, &w->map_wq_256, &w->map_wq_128, &w->map_l2_256,
              &w->map_l2_128, w->d_wsf, w->d_bias, w->alpha_w, Y_bf16, 0};
+  g.map_wsf = &w->map_wsf;
   g.err = d.err;
   return launch_gemm_w4a4(g, s);
 }

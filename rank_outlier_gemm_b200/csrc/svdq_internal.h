@@ -43,6 +43,9 @@ svdq_status check_device();
 svdq_status make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
                          uint64_t inner, uint64_t outer, uint64_t row_bytes, uint32_t box_inner,
                          uint32_t box_outer, CUtensorMapSwizzle swizzle);
+// 3-D tiled tensor map, no swizzle: dims[0] innermost, strides in bytes of dims 1 and 2.
+svdq_status make_tmap_3d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, const uint64_t dims[3],
+                         const uint64_t strides[2], const uint32_t box[3]);
 
 inline int round_up(int x, int m) { return (x + m - 1) / m * m; }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -83,6 +86,9 @@ struct GemmArgs {
   void* Y;                  // device bf16 [M, N]
   int ksplit;               // CTAs per output tile along K (0 = automatic, 1 = no split)
   int* err = nullptr;       // device error word (nullptr = the device's default word)
+  // weight scale atoms as [128-row blocks][64-element K blocks][128 x u32], box 4 K blocks x 2 row
+  // blocks (both halves of a 256-row tile in one copy); nullptr = the CTA-pair kernel is not used
+  const CUtensorMap* map_wsf = nullptr;
 };
 svdq_status launch_gemm_w4a4(const GemmArgs& a, cudaStream_t stream);
 
@@ -176,5 +182,6 @@ struct svdq_weights {
   // tensor maps over the weight-side buffers
   CUtensorMap map_l1{};
   CUtensorMap map_wq_256{}, map_wq_128{};
+  CUtensorMap map_wsf{};  // NVFP4 scale atoms, 3-D (see GemmArgs::map_wsf)
   CUtensorMap map_l2_256{}, map_l2_128{};
 };
