@@ -222,9 +222,12 @@ svdq_status svdq_quantize_act_lowrank_down(const svdq_weights* w, const void* X_
  * split over a cluster of up to 8 CTAs per tile and the fp32 partials are
  * summed in a fixed order through distributed shared memory; the result is
  * then deterministic but its rounding differs from the unsplit sum within
- * fp32 accumulation error.  The launch is a programmatic dependent of the
- * kernel ahead of it in the stream: it reads xq, xsf and T only once that
- * kernel has completed.
+ * fp32 accumulation error.  With many tiles and K > 3840 the tiles are
+ * 256 x 256 over clusters of two CTAs (one M = 256 MMA per K block, issued
+ * by one CTA of the pair); every output element is the same sum in the same
+ * order, so Y is bitwise the one-CTA result.  The launch is a programmatic
+ * dependent of the kernel ahead of it in the stream: it reads xq, xsf and T
+ * only once that kernel has completed.
  * For an INT4 handle the codes and scales are expanded on chip into fp16 tiles
  * (q * s with a bf16 s is exact in fp16 while |q s| stays in fp16's range)
  * and contracted by fp16 tensor-core MMAs:
@@ -385,7 +388,8 @@ svdq_status svdq_debug_launch_stalled_act(const svdq_weights* w, const void* X_b
 
 /*
  * Test hook: svdq_linear_w4a4 with the split-K factor fixed to `ksplit` CTAs
- * per output tile (1 = no split) instead of the automatic choice.  The split
+ * per output tile (1 = no split, one CTA per 128 x 256 tile and never the
+ * CTA pair) instead of the automatic choice.  The split
  * is clamped to the number of 256-wide K tiles; a split whose clusters would
  * not all be resident at once falls back to 1.  INT4 handles have no split-K:
  * for them the call is svdq_linear_w4a4.  SVDQ_ERR_INVALID_ARG unless
