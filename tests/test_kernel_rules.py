@@ -4,7 +4,9 @@
   wait that nothing completes ends with an error status instead of hanging;
 * no device code traps or asserts (a failure is reported through the device
   error word and the context stays usable);
-* every TMEM allocation in a kernel has a matching release in that kernel.
+* every TMEM allocation in a kernel has a matching release in that kernel;
+* no TMA or bulk copy uses cluster multicast (each CTA loads its own tiles;
+  only tcgen05.commit arrivals are multicast across a CTA pair).
 """
 
 import os
@@ -80,3 +82,16 @@ def test_tmem_allocations_are_released(name):
     allocs = len(re.findall(r"\btmem_alloc\w*\s*\(", src))
     frees = len(re.findall(r"\btmem_dealloc\w*\s*\(", src))
     assert allocs == frees
+
+
+@pytest.mark.parametrize("name", SOURCES)
+def test_no_multicast_copies(name):
+    src = open(os.path.join(CSRC, name)).read()
+    for line in src.splitlines():
+        if "cp.async.bulk" in line:
+            assert "multicast" not in line, f"{name}: multicast copy: {line.strip()}"
+
+
+def test_the_multicast_check_would_see_one():
+    planted = '"cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.multicast::cluster"'
+    assert "cp.async.bulk" in planted and "multicast" in planted
