@@ -84,14 +84,17 @@ def test_tmem_allocations_are_released(name):
     assert allocs == frees
 
 
+def _multicast_copies(src):
+    return [line.strip() for line in src.splitlines() if "cp.async.bulk" in line and "multicast" in line]
+
+
 @pytest.mark.parametrize("name", SOURCES)
 def test_no_multicast_copies(name):
-    src = open(os.path.join(CSRC, name)).read()
-    for line in src.splitlines():
-        if "cp.async.bulk" in line:
-            assert "multicast" not in line, f"{name}: multicast copy: {line.strip()}"
+    assert _multicast_copies(open(os.path.join(CSRC, name)).read()) == []
 
 
-def test_the_multicast_check_would_see_one():
-    planted = '"cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.multicast::cluster"'
-    assert "cp.async.bulk" in planted and "multicast" in planted
+def test_the_multicast_check_sees_a_planted_one():
+    planted = ('asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes'
+               '.multicast::cluster [%0], [%1, {%2, %3}], [%4], %5;" :: ...);\n'
+               'asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64");')
+    assert len(_multicast_copies(planted)) == 1
